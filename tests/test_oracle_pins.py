@@ -1,0 +1,365 @@
+"""Pins for the CPU oracle: each oracle step is checked against something other
+than itself -- a library routine (numpy's fp16 cast, transformers' RoPE,
+scipy's Hadamard matrix, torch fp64 attention), a closed form, an invariant
+the method relies on, or brute force on tiny inputs.
+
+Passages: "RotateAttention: RoPE-Aware Rotation and Range Rectification for
+INT4 Quantized Attention in Video Generation", abstract (3D RoPE,
+RoPE-aware rotation, INT4 FlashAttention, range-optimised P quantisation with
+fixed scale and zero-point, FP16 fallback).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from video_dit_b200 import synth
+
+
+# ------------------------------------------------------------ fp16 casts ---
+
+def test_half_to_float_exhaustive():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float32)
+    got = np.array([oracle.half_to_float(int(b)) for b in bits], np.float32)
+    finite = np.isfinite(ref)
+    assert np.array_equal(got[finite].view(np.uint32), ref[finite].view(np.uint32))
+    assert np.all(np.isnan(got[np.isnan(ref)]))
+    assert np.array_equal(np.isinf(got), np.isinf(ref))
+
+
+def test_float_to_half_rne_against_numpy():
+    rng = np.random.default_rng(0)
+    h = np.arange(0, 0x7bff, 7, dtype=np.uint16).view(np.float16).astype(np.float32)
+    # exact halves, midpoints between neighbours (ties), 1 fp32 ulp either side, randoms
+    nxt = np.nextafter(h.astype(np.float16), np.float16(np.inf)).astype(np.float32)
+    mid = ((h.astype(np.float64) + nxt.astype(np.float64)) / 2).astype(np.float32)
+    xs = np.concatenate([h, mid, np.nextafter(mid, np.float32(0)), np.nextafter(mid, np.float32(1e9)),
+                         rng.standard_normal(20000).astype(np.float32) * 30,
+                         rng.standard_normal(2000).astype(np.float32) * 1e-5,
+                         np.float32([65504, 65519.9, 65520, 1e6, 2.0 ** -25, 2.0 ** -24 * 1.5])])
+    xs = np.concatenate([xs, -xs])
+    with np.errstate(over="ignore"):
+        ref = xs.astype(np.float16).view(np.uint16)
+    got = np.array([oracle.float_to_half(float(x)) for x in xs], np.uint16)
+    assert np.array_equal(got, ref)
+
+
+# ------------------------------------------------------------------ RoPE ---
+
+def _hf_rope_axis(d_a, npos, theta):
+    from transformers import LlamaConfig
+    from transformers.models.llama.modeling_llama import LlamaRotaryEmbedding
+    cfg = LlamaConfig(hidden_size=d_a * 2, num_attention_heads=2, head_dim=d_a, rope_theta=theta)
+    emb = LlamaRotaryEmbedding(cfg)
+    pos = torch.arange(npos)[None]
+    cos, sin = emb(torch.zeros(1, npos, d_a, dtype=torch.float64), pos)
+    return cos[0].numpy(), sin[0].numpy()          # [npos, d_a], half-split layout
+
+
+@pytest.mark.parametrize("rope_dim,grid", [((16, 24, 24), (4, 8, 8)), ((44, 42, 42), (21, 30, 52)),
+                                           ((16, 56, 56), (33, 34, 60))])
+def test_rope_tables_match_transformers(rope_dim, grid):
+    c, s = oracle.rope_tables(grid, rope_dim)
+    off = 0
+    for a in range(3):
+        half = rope_dim[a] // 2
+        hc, hs = _hf_rope_axis(rope_dim[a], grid[a], 10000.0)
+        oc = c[off: off + grid[a] * half].reshape(grid[a], half)
+        os_ = s[off: off + grid[a] * half].reshape(grid[a], half)
+        # transformers' inv_freq is fp32, so angles agree to ~pos * 1e-7
+        assert np.abs(oc - hc[:, :half]).max() < 2e-5
+        assert np.abs(os_ - hs[:, :half]).max() < 2e-5
+        off += grid[a] * half
+
+
+def test_rope_row_matches_transformers_apply():
+    """Interleaved pairs (2i, 2i+1) of the oracle == transformers' half-split
+    rotate_half after the channel permutation (i, i + d_a/2) <- (2i, 2i+1)."""
+    from transformers.models.llama.modeling_llama import apply_rotary_pos_emb
+    rope_dim, grid = (44, 42, 42), (21, 30, 52)
+    rng = np.random.default_rng(1)
+    for n in [0, 1, 52, 1561, 32759, 17 * 1560 + 29 * 52 + 51]:
+        x = rng.standard_normal(128).astype(np.float32)
+        y = oracle.rope_rotate_row(x, n, grid, rope_dim, (1, 1, 1), rotate=False)
+        pos = (n // (30 * 52), (n // 52) % 30, n % 52)
+        off = 0
+        for a in range(3):
+            d_a = rope_dim[a]
+            hc, hs = _hf_rope_axis(d_a, grid[a], 10000.0)
+            part = x[off: off + d_a].astype(np.float64)
+            hf_in = np.concatenate([part[0::2], part[1::2]])
+            t = torch.from_numpy(hf_in)[None, None, None]
+            cos = torch.from_numpy(hc[pos[a]])[None, None]
+            sin = torch.from_numpy(hs[pos[a]])[None, None]
+            out, _ = apply_rotary_pos_emb(t, t, cos, sin)
+            out = out[0, 0, 0].numpy()
+            want = np.empty(d_a)
+            want[0::2], want[1::2] = out[: d_a // 2], out[d_a // 2:]
+            assert np.abs(y[off: off + d_a] - want).max() < 1e-4 * (1 + np.abs(want).max())
+            off += d_a
+
+
+def test_rope_identity_at_origin_and_relative_position():
+    rope_dim, grid = (16, 24, 24), (4, 8, 8)
+    rng = np.random.default_rng(2)
+    q = rng.standard_normal(64).astype(np.float32)
+    k = rng.standard_normal(64).astype(np.float32)
+    y = oracle.rope_rotate_row(q, 0, grid, rope_dim, (1, 1, 1), rotate=False)
+    assert np.array_equal(y, q)
+
+    def tok(t, h, w):
+        return (t * grid[1] + h) * grid[2] + w
+    # (t,h,w) pairs and a shift; dot products depend only on the offset
+    for (p1, p2, sh) in [((0, 0, 0), (1, 3, 5), (2, 4, 2)), ((1, 7, 2), (0, 1, 7), (1, 0, 0)),
+                         ((0, 2, 6), (3, 0, 0), (0, 3, 1))]:
+        a = np.dot(oracle.rope_rotate_row(q, tok(*p1), grid, rope_dim, (1, 1, 1), rotate=False),
+                   oracle.rope_rotate_row(k, tok(*p2), grid, rope_dim, (1, 1, 1), rotate=False))
+        s1 = tuple(x + s for x, s in zip(p1, sh))
+        s2 = tuple(x + s for x, s in zip(p2, sh))
+        b = np.dot(oracle.rope_rotate_row(q, tok(*s1), grid, rope_dim, (1, 1, 1), rotate=False),
+                   oracle.rope_rotate_row(k, tok(*s2), grid, rope_dim, (1, 1, 1), rotate=False))
+        assert abs(a - b) < 1e-4 * (1 + abs(a))
+
+
+# -------------------------------------------------------------- rotation ---
+
+@pytest.mark.parametrize("rope_dim,had", [((16, 24, 24), (16, 8, 8)), ((44, 42, 42), (4, 2, 2)),
+                                          ((16, 56, 56), (16, 8, 8)), ((44, 42, 42), (1, 1, 1))])
+def test_rotation_is_blockdiag_sylvester_hadamard(rope_dim, had):
+    from scipy.linalg import block_diag, hadamard
+    d = sum(rope_dim)
+    M = np.stack([oracle.rope_rotate_row(np.eye(d, dtype=np.float32)[j], 0, (1, 1, 1), rope_dim, had,
+                                         rope=False) for j in range(d)], axis=1)
+    blocks = []
+    for a in range(3):
+        b = had[a]
+        blocks += [hadamard(b) / math.sqrt(b)] * (rope_dim[a] // b)
+    want = block_diag(*blocks)
+    assert np.abs(M - want).max() <= 1e-7
+    assert np.abs(M @ M.T - np.eye(d)).max() < 1e-6
+
+
+def test_rotation_preserves_qk():
+    rope_dim, had = (44, 42, 42), (4, 2, 2)
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        q = (rng.standard_normal(128) * np.where(rng.random(128) < 0.05, 15, 1)).astype(np.float32)
+        k = rng.standard_normal(128).astype(np.float32)
+        rq = oracle.rope_rotate_row(q, 0, (1, 1, 1), rope_dim, had, rope=False)
+        rk = oracle.rope_rotate_row(k, 0, (1, 1, 1), rope_dim, had, rope=False)
+        ref = np.dot(q.astype(np.float64), k.astype(np.float64))
+        assert abs(np.dot(rq.astype(np.float64), rk.astype(np.float64)) - ref) < 1e-5 * (
+            np.abs(q).sum() * np.abs(k).max())
+
+
+# ------------------------------------------------------------- quantiser ---
+
+@pytest.mark.parametrize("amax", [1.0, 0.3, 7.0, 42.123, 65504.0, 3.1e-3])
+def test_quantiser_exhaustive_fp16(amax):
+    ys = np.arange(65536, dtype=np.uint32).astype(np.uint16).view(np.float16).astype(np.float32)
+    ys = ys[np.isfinite(ys) & (np.abs(ys) <= np.float32(amax))]
+    scale, inv = oracle.quant_params(amax)
+    assert scale == np.float32(amax) / np.float32(7) and inv == np.float32(7) / np.float32(amax)
+    c = oracle.quant_codes(ys, inv).astype(np.int64)
+    assert c.min() >= -7 and c.max() <= 7
+    # numpy's IEEE fp32 multiply and round-half-even give the same codes
+    assert np.array_equal(c, np.clip(np.rint(ys * np.float32(inv)), -7, 7).astype(np.int64))
+    err = np.abs(ys.astype(np.float64) - c * np.float64(scale))
+    assert err.max() <= np.float64(scale) / 2 * (1 + 2.0 ** -20)
+    order = np.argsort(ys, kind="stable")
+    assert np.all(np.diff(c[order]) >= 0)                     # monotone
+    assert oracle.quant_code(amax, inv) == 7 and oracle.quant_code(-amax, inv) == -7
+    assert np.array_equal(oracle.quant_codes(-ys, inv), -oracle.quant_codes(ys, inv))
+
+
+def test_quantiser_zero_block():
+    assert oracle.quant_params(0.0) == (0.0, 0.0)
+    assert oracle.quant_code(0.0, 0.0) == 0
+
+
+# --------------------------------------------------------------- P codes ---
+
+def _thresholds():
+    """tau_k: the smallest fp32 d with RNE(15 * 2^d) >= k, from mpmath at 60 digits."""
+    import mpmath
+    mpmath.mp.dps = 60
+    taus = {}
+    for k in range(1, 16):
+        t = mpmath.log((mpmath.mpf(k) - mpmath.mpf("0.5")) / 15, 2)
+        f = np.float32(float(t))
+        while mpmath.mpf(float(f)) < t:
+            f = np.nextafter(f, np.float32(1))
+        while mpmath.mpf(float(np.nextafter(f, np.float32(-10)))) >= t:
+            f = np.nextafter(f, np.float32(-10))
+        taus[k] = f
+    return taus
+
+
+def test_pcode_thresholds():
+    taus = _thresholds()
+    assert taus[8] == np.float32(-1.0)          # 15 * 2^-1 = 7.5 is the only tie: RNE -> 8
+    for k, t in taus.items():
+        assert oracle.pcode(float(t)) == k, (k, t)
+        assert oracle.pcode(float(np.nextafter(t, np.float32(-10)))) == k - 1, (k, t)
+    assert oracle.pcode(0.0) == 15
+    assert oracle.pcode(-0.0) == 15
+    assert oracle.pcode(-200.0) == 0
+    assert oracle.pcode(3e-8) == 15
+
+
+def test_pcode_dense_sample_matches_threshold_form():
+    taus = _thresholds()
+    tau = np.array([taus[k] for k in range(1, 16)], np.float32)
+    rng = np.random.default_rng(4)
+    d = np.concatenate([rng.uniform(-6, 0, 2_000_000).astype(np.float32),
+                        (tau[:, None] + np.arange(-64, 65)[None, :] * np.float32(2 ** -22)).ravel()])
+    d = d[d <= 0]
+    u = oracle.pcode_array(d)
+    want = np.searchsorted(tau, d, side="right")             # #{k: tau_k <= d}
+    assert np.array_equal(u.astype(np.int64), want)
+
+
+# ------------------------------------------------------ whole pipeline ---
+
+def _tiny(**kw):
+    w = synth.WORKLOADS["tiny"]
+    return synth.scaled(w, "tiny_pin", **kw) if kw else w
+
+
+def test_prepare_codes_reconstruct_rotated_values():
+    w = _tiny()
+    q, k, v = synth.make_inputs(w)
+    p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block)
+    for name, src in (("q", q), ("k", k)):
+        codes = oracle.unpack_s4(p[f"{name}_codes"][0, 1]).astype(np.float64)
+        scale = np.repeat(p[f"{name}_scale"][0, 1], 64).astype(np.float64)
+        for n in range(0, w.N, 37):
+            y = oracle.rope_rotate_row(src[0, 1, n].astype(np.float32), n, w.grid, w.rope_dim, w.had_block)
+            assert np.abs(codes[n] * scale[n] - y).max() <= scale[n] / 2 * (1 + 1e-6)
+        for j in range(w.N // 64):
+            assert np.abs(codes[j * 64:(j + 1) * 64]).max() == 7
+    vc = oracle.unpack_s4(p["v_codes"][0, 0]).astype(np.float64)       # [blk, d, 64]
+    vs = p["v_scale"][0, 0].astype(np.float64)                          # [blk, d]
+    deq = (vc * vs[:, :, None]).transpose(0, 2, 1).reshape(-1, w.d)
+    vv = v[0, 0].astype(np.float64)
+    assert np.all(np.abs(deq - vv) <= np.repeat(vs, 64, axis=0) / 2 * (1 + 1e-6))
+
+
+def test_integer_scores_brute_force():
+    w = _tiny()
+    q, k, v = synth.make_inputs(w)
+    p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block)
+    _, s, _ = oracle.attn_int4(p, w.N, 1 / math.sqrt(w.d), 0, 1, 0, w.N, dump=True)
+    qc = oracle.unpack_s4(p["q_codes"][0, 1]).astype(np.int64)
+    kc = oracle.unpack_s4(p["k_codes"][0, 1]).astype(np.int64)
+    assert np.array_equal(s, qc @ kc.T)
+
+
+def test_pcodes_span_full_range_and_offset_identity():
+    w = _tiny()
+    q, k, v = synth.make_inputs(w)
+    p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block)
+    hist = np.zeros(16, np.int64)
+    for h in range(w.H):
+        _, _, u = oracle.attn_int4(p, w.N, 1 / math.sqrt(w.d), 0, h, 0, w.N, dump=True)
+        hist += np.bincount(u.ravel(), minlength=16)
+        vc = oracle.unpack_s4(p["v_codes"][0, h]).astype(np.int64)    # [blk, d, 64]
+        for j in range(w.N // 64):
+            uj = u[:, j * 64:(j + 1) * 64].astype(np.int64)
+            lhs = uj @ vc[j].T
+            rhs = (uj - 8) @ vc[j].T + 8 * vc[j].sum(axis=1)[None, :]
+            assert np.array_equal(lhs, rhs)
+    assert np.all(hist > 0), hist          # unsigned codes use all 16 levels
+
+
+def test_online_and_closed_forms_agree():
+    w = synth.scaled(synth.WORKLOADS["wan480"], "mini", H=1, grid=(2, 5, 13))     # N = 130: ragged
+    q, k, v = synth.make_inputs(w)
+    p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block)
+    a = oracle.attn_int4(p, w.N, 1 / math.sqrt(w.d), 0, 0, 0, w.N, online=False)
+    b = oracle.attn_int4(p, w.N, 1 / math.sqrt(w.d), 0, 0, 0, w.N, online=True)
+    assert np.abs(a - b).max() < 1e-12 * (1 + np.abs(a).max())
+
+
+def test_uniform_attention_when_scores_vanish():
+    """Q = 0 -> every score is 0 -> every P code is 15 -> the output is the
+    mean of the dequantised V rows."""
+    w = synth.scaled(synth.WORKLOADS["wan480"], "zeroq", H=1, grid=(1, 5, 20))     # N = 100
+    q, k, v = synth.make_inputs(w)
+    q[:] = 0
+    p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block)
+    out, _, u = oracle.attn_int4(p, w.N, 1 / math.sqrt(w.d), 0, 0, 0, w.N, dump=True)
+    assert np.all(u == 15)
+    vc = oracle.unpack_s4(p["v_codes"][0, 0]).astype(np.float64)
+    deq = (vc * p["v_scale"][0, 0].astype(np.float64)[:, :, None]).transpose(0, 2, 1).reshape(-1, w.d)
+    assert np.abs(out - deq[: w.N].mean(axis=0)[None]).max() < 1e-12
+
+
+def test_dominant_key_selects_its_value_row():
+    w = synth.scaled(synth.WORKLOADS["wan480"], "dom", H=1, grid=(1, 4, 32), qk_outliers=(0, 0, 0))
+    q, k, v = synth.make_inputs(w)
+    j = 10       # in the first key group: later groups are all coded against its max
+    k[0, 0, j] = np.float16(0)
+    k[0, 0, j, ::3] = np.float16(6)
+    q[0, 0, :] = np.float16(0)
+    q[0, 0, :, ::3] = np.float16(6)        # RoPE is position dependent: keep only row j's own token
+    p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block)
+    out, s, u = oracle.attn_int4(p, w.N, 1 / math.sqrt(w.d), 0, 0, j, 1, dump=True)
+    assert u[0, j] == 15 and u[0].sum() == 15
+    vc = oracle.unpack_s4(p["v_codes"][0, 0]).astype(np.float64)
+    row = vc[j // 64, :, j % 64] * p["v_scale"][0, 0, j // 64].astype(np.float64)
+    assert np.abs(out[0] - row).max() < 1e-12
+
+
+def test_single_group_is_global_max():
+    """group >= N: every P code is taken against the final row max."""
+    w = synth.scaled(synth.WORKLOADS["wan480"], "glob", H=1, grid=(2, 5, 13))
+    q, k, v = synth.make_inputs(w)
+    p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block)
+    out, s, u = oracle.attn_int4(p, w.N, 1 / math.sqrt(w.d), 0, 0, 0, w.N, group=1 << 20, dump=True)
+    assert np.all(u.max(axis=1) == 15)
+    kappa = np.float32(np.float64(np.float32(1 / math.sqrt(w.d))) * 1.4426950408889634)
+    qs = np.repeat(p["q_scale"][0, 0], 64)[: w.N]
+    ks = np.repeat(p["k_scale"][0, 0], 64)[: w.N]
+    c = (qs[:, None] * ks[None, :]).astype(np.float32) * kappa
+    x = s.astype(np.float32) * c
+    M = x.max(axis=1, keepdims=True)
+    dd = (s.astype(np.float64) * c.astype(np.float64) - M).astype(np.float32)  # one rounding
+    assert np.array_equal(u, oracle.pcode_array(dd))
+    vc = oracle.unpack_s4(p["v_codes"][0, 0]).astype(np.float64)
+    deq = (vc * p["v_scale"][0, 0].astype(np.float64)[:, :, None]).transpose(0, 2, 1).reshape(-1, w.d)
+    want = (u.astype(np.float64) @ deq[: w.N]) / u.sum(axis=1, keepdims=True)
+    assert np.abs(out - want).max() < 1e-12
+
+
+def test_fp16_path_matches_torch_sdpa_float64():
+    w = synth.scaled(synth.WORKLOADS["wan480"], "f16", H=2, grid=(2, 5, 13))
+    q, k, v = synth.make_inputs(w)
+    flags = np.ones(w.H, np.uint8)
+    p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block, flags=flags)
+    qr = torch.from_numpy(p["q_rope"].view(np.float16).astype(np.float64))
+    kr = torch.from_numpy(p["k_rope"].view(np.float16).astype(np.float64))
+    vv = torch.from_numpy(v.astype(np.float64))
+    sm = float(np.float32(1 / math.sqrt(w.d)))       # the oracle takes sm_scale as fp32
+    ref = torch.nn.functional.scaled_dot_product_attention(qr, kr, vv, scale=sm).numpy()
+    for h in range(w.H):
+        out = oracle.attn_fp16(p["q_rope"], p["k_rope"], v, 1 / math.sqrt(w.d), 0, h, 0, w.N)
+        assert np.abs(out - ref[0, h]).max() < 1e-12
+    # q_rope is the fp16 rounding of the RoPE'd row
+    for n in (0, 5, 129):
+        y = oracle.rope_rotate_row(q[0, 1, n].astype(np.float32), n, w.grid, w.rope_dim, w.had_block,
+                                   rotate=False)
+        assert np.array_equal(p["q_rope"][0, 1, n], y.astype(np.float16).view(np.uint16))
+
+
+def test_int4_close_to_unquantised_attention_on_plain_gaussians():
+    w = synth.scaled(synth.WORKLOADS["tiny"], "plain", qk_outliers=(0, 0, 0))
+    q, k, v = synth.make_inputs(w)
+    p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block)
+    out = oracle.attn_int4(p, w.N, 1 / math.sqrt(w.d), 0, 0, 0, w.N)
+    ref = oracle.attn_ref(q, k, v, w.grid, w.rope_dim, 1 / math.sqrt(w.d), 0, 0, 0, w.N)
+    cos = (out * ref).sum(1) / np.linalg.norm(out, axis=1) / np.linalg.norm(ref, axis=1)
+    assert cos.mean() > 0.93 and cos.min() > 0.75
