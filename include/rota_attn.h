@@ -1,0 +1,202 @@
+/*
+ * rota_attn.h -- C ABI of the B200 (sm_100a) RotateAttention forward.
+ *
+ * The method: "RotateAttention: RoPE-Aware Rotation and Range Rectification
+ * for INT4 Quantized Attention in Video Generation" (abstract and Key
+ * Points): a mixed-precision INT4 FlashAttention for DiT video models with 3D
+ * RoPE.  Q and K get 3D RoPE and then a RoPE-aware rotation (an orthogonal
+ * matrix inside each RoPE partition, which leaves Q K^T unchanged) before
+ * INT4 quantisation; P = exp(QK - max QK) is quantised with a fixed scale and
+ * zero-point that use the whole unsigned 4-bit range; heads or denoising
+ * steps flagged as accuracy-sensitive take an FP16 attention instead.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers allocated by the caller, except
+ *     where a parameter is marked "host".  The library never allocates,
+ *     never frees and never synchronises (except rota_attn_get_error).
+ *   - fp16 tensors are passed as their uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream); every
+ *     device call is enqueued asynchronously on it.
+ *   - Argument errors are detected on the host and returned synchronously,
+ *     with nothing enqueued.  Faults detected on the device (a bounded wait
+ *     that ran out, a failed bounds check) are recorded in a device error
+ *     word and reported by rota_attn_get_error.
+ *   - Layouts are row-major with the last index fastest; s4 codes are packed
+ *     two per byte, low nibble first, two's complement.
+ *   - Npad = 64 * ceil(N / 64); nblk = Npad / 64.
+ */
+#ifndef ROTA_ATTN_H
+#define ROTA_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ROTA_OK = 0,
+  ROTA_ERR_INVALID_ARG = 1,  /* a descriptor field, pointer, size or alignment is invalid */
+  ROTA_ERR_UNSUPPORTED = 2,  /* valid, but outside what the kernels implement (e.g. head_dim) */
+  ROTA_ERR_CUDA = 3,         /* a CUDA runtime call failed (launch, symbol copy, sync) */
+  ROTA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out; the context stays usable */
+  ROTA_ERR_DEVICE = 5        /* a device-side consistency check failed */
+} rota_status;
+
+/*
+ * Problem descriptor.  Token n of the sequence sits at grid position
+ * t = n / (grid_h * grid_w), h = (n / grid_w) % grid_h, w = n % grid_w
+ * (t-major raster), N == grid_t * grid_h * grid_w.
+ * rope_dim: channels of the temporal / height / width RoPE partitions, in
+ *   that order at channel offsets 0, rope_dim[0], rope_dim[0]+rope_dim[1];
+ *   each even, summing to head_dim (e.g. 44/42/42, 16/56/56, 16/24/24).
+ * had_block: size of the Hadamard blocks of the rotation inside each
+ *   partition: a power of two (1 = no rotation) dividing rope_dim[a], <= 64.
+ * rope_theta: RoPE base (10000).
+ * sm_scale: softmax scale; 0 selects 1/sqrt(head_dim) (rounded to fp32).
+ * head_dim: 64 or 128.
+ */
+typedef struct {
+  int32_t B, H, N, head_dim;
+  int32_t grid_t, grid_h, grid_w;
+  int32_t rope_dim[3];
+  int32_t had_block[3];
+  float rope_theta;
+  float sm_scale;
+} rota_attn_desc;
+
+/*
+ * Caller-owned device buffers written by rota_attn_prepare_qk and read by the
+ * attention calls (sizes from rota_attn_buffer_sizes; every pointer 16-byte
+ * aligned):
+ *   q_codes, k_codes : uint8 [B,H,Npad,head_dim/2]  rotated, RoPE'd Q/K codes
+ *   q_scale, k_scale : fp32  [B,H,nblk]               one scale per 64 tokens
+ *   v_codes          : uint8 [B,H,nblk,head_dim,32]  64 tokens of one channel
+ *   v_scale          : fp32  [B,H,nblk,head_dim]     per channel per 64 tokens
+ *   q_rope, k_rope   : fp16  [B,H,N,head_dim]        RoPE'd Q/K of flagged heads
+ *                      (may be NULL when no head is flagged)
+ *   rope_cos, rope_sin: fp32 tables from rota_attn_build_rope_tables, copied
+ *                      to the device by the caller.
+ */
+typedef struct {
+  uint8_t* q_codes;
+  uint8_t* k_codes;
+  float* q_scale;
+  float* k_scale;
+  uint8_t* v_codes;
+  float* v_scale;
+  uint16_t* q_rope;
+  uint16_t* k_rope;
+  const float* rope_cos;
+  const float* rope_sin;
+} rota_attn_buffers;
+
+/* Indices into the `bytes` array of rota_attn_buffer_sizes. */
+enum {
+  ROTA_BUF_Q_CODES = 0,
+  ROTA_BUF_K_CODES,
+  ROTA_BUF_Q_SCALE,
+  ROTA_BUF_K_SCALE,
+  ROTA_BUF_V_CODES,
+  ROTA_BUF_V_SCALE,
+  ROTA_BUF_Q_ROPE,
+  ROTA_BUF_K_ROPE,
+  ROTA_BUF_ROPE_TABLE, /* each of rope_cos and rope_sin */
+  ROTA_BUF_COUNT
+};
+
+/* Checks a descriptor (fills nothing).  ROTA_ERR_INVALID_ARG with no side effects. */
+rota_status rota_attn_validate(const rota_attn_desc* desc);
+
+/* Host: byte size of each buffer (array of ROTA_BUF_COUNT entries, host). */
+rota_status rota_attn_buffer_sizes(const rota_attn_desc* desc, size_t* bytes);
+
+/*
+ * Host: the 3D RoPE tables (3D RoPE of the abstract; RoFormer frequencies
+ * restarted per partition).  For axis a (t, h, w) of extent P_a and
+ * partition d_a, entry [pos][i] (i < d_a/2) holds cos / sin of
+ * pos * rope_theta^(-2i/d_a), evaluated in double and rounded to fp32.  Axes
+ * are concatenated t, h, w.  host_cos / host_sin: host arrays of
+ * bytes[ROTA_BUF_ROPE_TABLE] / 4 floats.
+ */
+rota_status rota_attn_build_rope_tables(const rota_attn_desc* desc, float* host_cos, float* host_sin);
+
+/*
+ * The prologue (3D RoPE -> RoPE-aware rotation -> INT4 quantisation; the two
+ * techniques of the abstract's pipeline up to the attention), one launch.
+ *   q, k, v         : fp16 [B,H,N,head_dim] device inputs (after the QKV projection)
+ *   head_flags      : host uint8 [H]; 1 = the head takes the FP16 fallback at this
+ *                     call (per head, per denoising step), 0 = INT4.  NULL = all INT4.
+ * INT4 heads: Q and K get RoPE (fp32, pair (2i, 2i+1) of each partition
+ *   rotated by the table angle), then the normalised Sylvester Hadamard H_b/sqrt(b)
+ *   on consecutive blocks of had_block[a] channels inside each partition, then
+ *   symmetric INT4 codes, one scale per 64 tokens x head_dim block:
+ *   scale = amax/7, code = clamp(rne(y * (7/amax)), -7, 7).  V (no RoPE, no
+ *   rotation) gets the same quantiser per channel per 64-token block.  Tokens
+ *   >= N get code 0 and no weight in any amax.
+ * FP16 heads: q_rope / k_rope = fp16(RoPE(q)), fp16(RoPE(k)); no codes.
+ */
+rota_status rota_attn_prepare_qk(const rota_attn_desc* desc, const uint16_t* q, const uint16_t* k,
+                                 const uint16_t* v, const uint8_t* head_flags,
+                                 const rota_attn_buffers* buf, void* stream);
+
+/*
+ * INT4 attention (the abstract's mixed-precision INT4 FlashAttention) for the
+ * heads whose flag is 0.  Integer Q K^T on the tensor cores (s32); scores
+ * dequantised with c = (sq * sk) * (sm_scale * log2 e); a running max m over
+ * consecutive 64-key groups; range-optimised P codes u = rne(15 * 2^(S c - m))
+ * in 0..15 (fixed scale 1/15, zero-point 0: the whole unsigned 4-bit range,
+ * as the abstract's "Range-optimized P Quantization" asks); integer P V on
+ * the tensor cores per 64-key block; V scales, rescaling by 2^(m_old - m_new)
+ * and the row sum of the codes in fp32; out = O / l.
+ *   out: fp32 [B,H,N,head_dim]; rows of flagged heads are not written.
+ */
+rota_status rota_attn_fwd_int4(const rota_attn_desc* desc, const rota_attn_buffers* buf,
+                               const uint8_t* head_flags, float* out, void* stream);
+
+/*
+ * FP16 fallback (the abstract's "selective FP16 fallback") for the heads whose
+ * flag is 1: softmax(sm_scale * q_rope k_rope^T) v with fp16 tensor-core
+ * products, fp32 accumulation and an fp32 online softmax.
+ *   v  : the fp16 V input of rota_attn_prepare_qk;  out: fp32 [B,H,N,head_dim]
+ *   (rows of unflagged heads are not written).
+ */
+rota_status rota_attn_fwd_fp16_fallback(const rota_attn_desc* desc, const rota_attn_buffers* buf,
+                                        const uint16_t* v, const uint8_t* head_flags, float* out,
+                                        void* stream);
+
+/* Synchronises `stream`, then returns and clears the device error word
+ * (ROTA_OK, ROTA_ERR_TIMEOUT or ROTA_ERR_DEVICE), or ROTA_ERR_CUDA if the
+ * synchronisation itself failed. */
+rota_status rota_attn_get_error(void* stream);
+
+/* Static string for a status code. */
+const char* rota_attn_status_string(rota_status s);
+
+/* ---------------------------------------------------------- test hooks --- */
+
+/*
+ * Runs the INT4 attention kernel for head (b, h) only, with its debug dump
+ * enabled: for rows [r0, r0+nr) it also stores the s32 scores S (device int32
+ * [nr, N]) and the P codes (device uint8 [nr, N]).  `out` as for
+ * rota_attn_fwd_int4 (only that head's rows are written).
+ */
+rota_status rota_attn_debug_dump_int4(const rota_attn_desc* desc, const rota_attn_buffers* buf, int32_t b,
+                                      int32_t h, int32_t r0, int32_t nr, int32_t* s_out, uint8_t* p_out,
+                                      float* out, void* stream);
+
+/* Applies the kernels' P-code function to n exponents d (device fp32 ->
+ * device uint8), so it can be checked exhaustively against the definition. */
+rota_status rota_attn_debug_pcode(const float* d, uint8_t* u, int64_t n, void* stream);
+
+/* Fault injection for the bounded waits: the next INT4 launch skips its first
+ * score MMA, so every wait on it runs out after `timeout_ns` and the kernel
+ * exits with ROTA_ERR_TIMEOUT.  One-shot; 0 disarms. */
+rota_status rota_attn_debug_inject_timeout(int32_t arm, uint64_t timeout_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROTA_ATTN_H */

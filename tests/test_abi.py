@@ -1,0 +1,108 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports
+every function include/rota_attn.h declares, rejects bad arguments before
+touching the device, and its host-built RoPE tables equal the oracle's byte
+for byte."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from video_dit_b200 import build as vbuild
+from video_dit_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def ra():
+    vbuild.build()
+    from video_dit_b200 import rota_attn
+    return rota_attn
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "rota_attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(rota_attn_\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(ra):
+    names = declared_functions()
+    assert len(names) >= 11
+    lib = ctypes.CDLL(ra.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def _desc(ra, w):
+    return ra.make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta)
+
+
+def test_validate_accepts_workloads(ra):
+    for w in synth.WORKLOADS.values():
+        assert ra.rota_attn_validate(_desc(ra, w)) == ra.ROTA_OK, w.name
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("N", 1000, 1), ("head_dim", 96, 1), ("B", 0, 1), ("grid_w", 0, 1),
+    ("rope_theta", -1.0, 1), ("sm_scale", float("nan"), 1), ("H", 300, 2),
+])
+def test_validate_rejects(ra, field, value, status):
+    d = _desc(ra, synth.WORKLOADS["wan480"])
+    setattr(d, field, value)
+    assert ra.rota_attn_validate(d) == status
+
+
+def test_validate_rejects_bad_partitions(ra):
+    d = _desc(ra, synth.WORKLOADS["wan480"])
+    d.rope_dim[:] = [43, 43, 42]
+    assert ra.rota_attn_validate(d) == ra.ROTA_ERR_INVALID_ARG
+    d = _desc(ra, synth.WORKLOADS["wan480"])
+    d.had_block[:] = [8, 2, 2]                  # 8 does not divide 44
+    assert ra.rota_attn_validate(d) == ra.ROTA_ERR_INVALID_ARG
+    d.had_block[:] = [3, 2, 2]
+    assert ra.rota_attn_validate(d) == ra.ROTA_ERR_INVALID_ARG
+    d = _desc(ra, synth.WORKLOADS["tiny"])
+    d.head_dim = 128                             # partitions sum to 64
+    assert ra.rota_attn_validate(d) == ra.ROTA_ERR_INVALID_ARG
+
+
+def test_null_arguments_rejected_on_host(ra):
+    d = _desc(ra, synth.WORKLOADS["tiny"])
+    b = ra.rota_attn_buffers()
+    assert ra._lib.rota_attn_prepare_qk(ctypes.byref(d), None, None, None, None, ctypes.byref(b), None) == 1
+    assert ra._lib.rota_attn_fwd_int4(ctypes.byref(d), ctypes.byref(b), None, None, None) == 1
+    assert ra._lib.rota_attn_fwd_fp16_fallback(ctypes.byref(d), ctypes.byref(b), None, None, None, None) == 1
+    assert ra._lib.rota_attn_debug_pcode(None, None, 5, None) == 1
+    assert ra._lib.rota_attn_prepare_qk(None, None, None, None, None, None, None) == 1
+    assert ra.rota_attn_status_string(4) == "device wait timed out"
+
+
+def test_buffer_sizes(ra):
+    w = synth.WORKLOADS["wan480"]
+    sz = ra.rota_attn_buffer_sizes(_desc(ra, w))
+    npad = 32768
+    assert sz[ra.ROTA_BUF_Q_CODES] == 40 * npad * 64
+    assert sz[ra.ROTA_BUF_V_CODES] == 40 * 512 * 128 * 32
+    assert sz[ra.ROTA_BUF_V_SCALE] == 40 * 512 * 128 * 4
+    assert sz[ra.ROTA_BUF_Q_ROPE] == 40 * 32760 * 128 * 2
+    assert sz[ra.ROTA_BUF_ROPE_TABLE] == 4 * (21 * 22 + 30 * 21 + 52 * 21)
+
+
+@pytest.mark.parametrize("name", ["tiny", "wan480", "wan720", "hunyuan"])
+def test_rope_tables_identical_to_oracle(ra, name):
+    w = synth.WORKLOADS[name]
+    c, s = ra.rota_attn_build_rope_tables(_desc(ra, w))
+    oc, os_ = oracle.rope_tables(w.grid, w.rope_dim, w.theta)
+    assert np.array_equal(c.view(np.uint32), oc.view(np.uint32))
+    assert np.array_equal(s.view(np.uint32), os_.view(np.uint32))
+
+
+def test_kappa_matches_oracle_definition(ra):
+    # the oracle's kappa: RN(RN(1/sqrt(d)) * log2 e) from double
+    for d in (64, 128):
+        sm = np.float32(1 / np.sqrt(d))
+        assert ra.kappa(d) == np.float32(np.float64(sm) * 1.4426950408889634074)

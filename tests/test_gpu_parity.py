@@ -1,0 +1,117 @@
+"""GPU parity: the CUDA path against the CPU oracle on the same seeded inputs.
+
+Bars: integer codes, scales, RoPE'd fp16 rows, s32 scores and P codes
+bit-exact; attention outputs within max-abs 2e-3 of the oracle's double
+result.  Sizes span several 128-row tiles and 64-key blocks with a ragged
+tail (N mod 64 != 0), both head dims (64, 128) and all three RoPE splits."""
+import numpy as np
+import pytest
+
+import oracle
+from video_dit_b200 import synth
+
+from gpu_util import row_stats, run, sm_scale
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+CASES = {
+    "tiny": synth.WORKLOADS["tiny"],                                                  # N=256, d=64
+    "wan_mini": synth.scaled(synth.WORKLOADS["wan480"], "wan_mini", H=3, grid=(3, 10, 13)),     # N=390
+    "hunyuan_mini": synth.scaled(synth.WORKLOADS["hunyuan"], "hy_mini", H=2, grid=(3, 9, 20)),  # N=540
+    "ragged_small": synth.scaled(synth.WORKLOADS["wan480"], "ragged", H=1, grid=(1, 3, 7)),     # N=21 < 64
+}
+
+
+def _oracle(w, q, k, v, flags=None):
+    return oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block, w.theta, flags)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_prologue_codes_bit_exact(name):
+    w = CASES[name]
+    q, k, v = synth.make_inputs(w)
+    codes, _, _ = run(w, q, k, v)
+    ref = _oracle(w, q, k, v)
+    for key in ("q_codes", "k_codes", "v_codes"):
+        assert np.array_equal(codes[key], ref[key]), key
+    for key in ("q_scale", "k_scale", "v_scale"):
+        assert np.array_equal(codes[key].view(np.uint32), ref[key].view(np.uint32)), key
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_int4_scores_and_pcodes_bit_exact(name):
+    w = CASES[name]
+    q, k, v = synth.make_inputs(w)
+    h = w.H - 1
+    r0, nr = (0, w.N) if w.N <= 400 else (w.N - 150, 150)
+    _, out, (s, p, _) = run(w, q, k, v, dump=(0, h, r0, nr))
+    ref = _oracle(w, q, k, v)
+    o_ref, s_ref, p_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, r0, nr, dump=True)
+    assert np.array_equal(s, s_ref)
+    assert np.array_equal(p, p_ref)
+    e, rel, cos = row_stats(out[0, h, r0:r0 + nr], o_ref)
+    assert e <= TOL, (e, rel, cos)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_int4_output_all_heads(name):
+    w = CASES[name]
+    q, k, v = synth.make_inputs(w)
+    _, out, _ = run(w, q, k, v)
+    ref = _oracle(w, q, k, v)
+    for h in range(w.H):
+        o_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, 0, w.N)
+        e, rel, cos = row_stats(out[0, h], o_ref)
+        assert e <= TOL, (h, e, rel, cos)
+
+
+@pytest.mark.parametrize("name", ["tiny", "wan_mini", "ragged_small"])
+def test_fp16_fallback_heads(name):
+    w = CASES[name]
+    q, k, v = synth.make_inputs(w)
+    flags = np.zeros(w.H, np.uint8)
+    flags[0] = 1
+    codes, out, _ = run(w, q, k, v, flags=flags)
+    ref = _oracle(w, q, k, v, flags)
+    assert np.array_equal(codes["q_rope"][0, 0], ref["q_rope"][0, 0])
+    assert np.array_equal(codes["k_rope"][0, 0], ref["k_rope"][0, 0])
+    o16 = oracle.attn_fp16(ref["q_rope"], ref["k_rope"], v, sm_scale(w), 0, 0, 0, w.N)
+    e, rel, cos = row_stats(out[0, 0], o16)
+    assert e <= TOL, (e, rel, cos)
+    for h in range(1, w.H):          # the INT4 heads of the same call are unaffected
+        o_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, 0, w.N)
+        assert row_stats(out[0, h], o_ref)[0] <= TOL
+
+
+def test_pcode_function_matches_oracle_dense():
+    import torch
+    from gpu_util import lib
+    ra = lib()
+    rng = np.random.default_rng(0)
+    d = np.concatenate([rng.uniform(-6, 0, 4_000_000).astype(np.float32),
+                        np.float32([-1.0, 0.0, -0.0, -5.0, -4.906890, -30.0, 1e-7])])
+    dd = torch.from_numpy(d).cuda()
+    u = torch.empty(d.size, dtype=torch.uint8, device="cuda")
+    ra._check(ra.rota_attn_debug_pcode(dd, u), "pcode")
+    assert np.array_equal(u.cpu().numpy(), oracle.pcode_array(d))
+
+
+def test_pcode_function_exhaustive_near_thresholds():
+    """Every fp32 within 2^16 ulps of each of the 15 code thresholds."""
+    import torch
+    from gpu_util import lib
+    ra = lib()
+    taus = []
+    for kk in range(1, 16):
+        x = np.float32(np.log2((kk - 0.5) / 15))
+        taus.append(x)
+    base = np.array(taus, np.float32).view(np.int32)
+    offs = np.arange(-(1 << 16), 1 << 16, dtype=np.int32)
+    d = (base[:, None] + offs[None, :]).ravel().view(np.float32)
+    d = d[d <= 0]
+    dd = torch.from_numpy(d).cuda()
+    u = torch.empty(d.size, dtype=torch.uint8, device="cuda")
+    ra._check(ra.rota_attn_debug_pcode(dd, u), "pcode")
+    assert np.array_equal(u.cpu().numpy(), oracle.pcode_array(d))

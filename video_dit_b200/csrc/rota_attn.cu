@@ -1,0 +1,383 @@
+// rota_attn.cu -- the C ABI (include/rota_attn.h): argument checks, the
+// host-side tables (3D RoPE angles, exact P-code thresholds) and the kernel
+// launches.  Builds into librota_attn.so with the three kernels
+// (prologue, INT4 attention, FP16 fallback).
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "../../include/rota_attn.h"
+#include "attn_fp16.cuh"
+#include "attn_int4.cuh"
+#include "prologue.cuh"
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per mbarrier wait
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int npad_of(int N) { return ((N + 63) / 64) * 64; }
+
+float sm_scale_of(const rota_attn_desc* d) {
+  return d->sm_scale > 0.f ? d->sm_scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(d->head_dim)));
+}
+
+// kappa = RN(sm_scale * log2 e): scores are dequantised straight into base-2 exponents.
+float kappa_of(const rota_attn_desc* d) {
+  return static_cast<float>(static_cast<double>(sm_scale_of(d)) * 1.44269504088896340736);
+}
+
+// tau[k] (k = 1..15): the smallest fp32 d with rne(15 * 2^d) >= k, i.e. with
+// 15 * 2^d >= k - 1/2 (ties only occur at k = 8, d = -1, and round up to the
+// even code 8).  Found by rounding log2((k - 1/2) / 15) to fp32 and stepping
+// one ulp at a time against a long-double evaluation.
+struct TauTable {
+  float tau[16];
+  TauTable() {
+    tau[0] = -INFINITY;
+    for (int k = 1; k <= 15; ++k) {
+      const long double target = (static_cast<long double>(k) - 0.5L) / 15.0L;
+      auto reaches = [&](float d) { return exp2l(static_cast<long double>(d)) >= target; };
+      float f = static_cast<float>(log2l(target));
+      while (!reaches(f)) f = nextafterf(f, INFINITY);
+      while (reaches(nextafterf(f, -INFINITY))) f = nextafterf(f, -INFINITY);
+      tau[k] = f;
+    }
+  }
+};
+
+const TauTable& tau_table() {
+  static const TauTable t;
+  return t;
+}
+
+struct Injection {
+  std::mutex mu;
+  int armed = 0;
+  uint64_t timeout_ns = kDefaultTimeoutNs;
+} g_inject;
+
+rota_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return ROTA_OK;
+  std::fprintf(stderr, "rota_attn: CUDA error: %s\n", cudaGetErrorString(e));
+  return ROTA_ERR_CUDA;
+}
+
+template <typename K>
+rota_status set_smem(K kernel, int bytes) {
+  return cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Heads with flag == want, written to `heads`; returns their count.
+int select_heads(const rota_attn_desc* d, const uint8_t* flags, int want, int16_t* heads) {
+  int n = 0;
+  for (int h = 0; h < d->H; ++h) {
+    const int f = flags ? (flags[h] ? 1 : 0) : 0;
+    if (f == want) heads[n++] = static_cast<int16_t>(h);
+  }
+  return n;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rota_attn_status_string(rota_status s) {
+  switch (s) {
+    case ROTA_OK: return "ok";
+    case ROTA_ERR_INVALID_ARG: return "invalid argument";
+    case ROTA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ROTA_ERR_CUDA: return "CUDA runtime error";
+    case ROTA_ERR_TIMEOUT: return "device wait timed out";
+    case ROTA_ERR_DEVICE: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+rota_status rota_attn_validate(const rota_attn_desc* d) {
+  if (!d) return ROTA_ERR_INVALID_ARG;
+  if (d->B < 1 || d->H < 1 || d->N < 1 || d->head_dim < 1) return ROTA_ERR_INVALID_ARG;
+  if (d->grid_t < 1 || d->grid_h < 1 || d->grid_w < 1) return ROTA_ERR_INVALID_ARG;
+  if (static_cast<long long>(d->grid_t) * d->grid_h * d->grid_w != d->N) return ROTA_ERR_INVALID_ARG;
+  int sum = 0;
+  for (int a = 0; a < 3; ++a) {
+    if (d->rope_dim[a] < 2 || d->rope_dim[a] % 2) return ROTA_ERR_INVALID_ARG;
+    if (!is_pow2(d->had_block[a]) || d->had_block[a] > 64 || d->rope_dim[a] % d->had_block[a])
+      return ROTA_ERR_INVALID_ARG;
+    sum += d->rope_dim[a];
+  }
+  if (sum != d->head_dim) return ROTA_ERR_INVALID_ARG;
+  if (!(d->rope_theta > 0.f) || !std::isfinite(d->rope_theta)) return ROTA_ERR_INVALID_ARG;
+  if (!(d->sm_scale >= 0.f) || !std::isfinite(d->sm_scale)) return ROTA_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128) return ROTA_ERR_UNSUPPORTED;
+  if (d->H > 256) return ROTA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(d->B) * d->H * npad_of(d->N) * d->head_dim > (1ll << 40)) return ROTA_ERR_UNSUPPORTED;
+  if (d->B > 65535) return ROTA_ERR_UNSUPPORTED;
+  return ROTA_OK;
+}
+
+rota_status rota_attn_buffer_sizes(const rota_attn_desc* d, size_t* bytes) {
+  const rota_status st = rota_attn_validate(d);
+  if (st != ROTA_OK) return st;
+  if (!bytes) return ROTA_ERR_INVALID_ARG;
+  const size_t heads = static_cast<size_t>(d->B) * d->H;
+  const size_t npad = npad_of(d->N), nblk = npad / 64, D = d->head_dim;
+  bytes[ROTA_BUF_Q_CODES] = heads * npad * D / 2;
+  bytes[ROTA_BUF_K_CODES] = heads * npad * D / 2;
+  bytes[ROTA_BUF_Q_SCALE] = heads * nblk * 4;
+  bytes[ROTA_BUF_K_SCALE] = heads * nblk * 4;
+  bytes[ROTA_BUF_V_CODES] = heads * nblk * D * 32;
+  bytes[ROTA_BUF_V_SCALE] = heads * nblk * D * 4;
+  bytes[ROTA_BUF_Q_ROPE] = heads * d->N * D * 2;
+  bytes[ROTA_BUF_K_ROPE] = heads * d->N * D * 2;
+  bytes[ROTA_BUF_ROPE_TABLE] = 4 * (static_cast<size_t>(d->grid_t) * (d->rope_dim[0] / 2) +
+                                    static_cast<size_t>(d->grid_h) * (d->rope_dim[1] / 2) +
+                                    static_cast<size_t>(d->grid_w) * (d->rope_dim[2] / 2));
+  return ROTA_OK;
+}
+
+rota_status rota_attn_build_rope_tables(const rota_attn_desc* d, float* host_cos, float* host_sin) {
+  const rota_status st = rota_attn_validate(d);
+  if (st != ROTA_OK) return st;
+  if (!host_cos || !host_sin) return ROTA_ERR_INVALID_ARG;
+  const int extent[3] = {d->grid_t, d->grid_h, d->grid_w};
+  const double theta = static_cast<double>(d->rope_theta);
+  size_t base = 0;
+  for (int a = 0; a < 3; ++a) {
+    const int half = d->rope_dim[a] / 2;
+    for (int i = 0; i < half; ++i) {
+      // omega_i = theta^(-2i / d_a), evaluated in double
+      const double omega = std::pow(theta, -static_cast<double>(2 * i) / static_cast<double>(d->rope_dim[a]));
+      for (int pos = 0; pos < extent[a]; ++pos) {
+        const double angle = static_cast<double>(pos) * omega;
+        host_cos[base + static_cast<size_t>(pos) * half + i] = static_cast<float>(std::cos(angle));
+        host_sin[base + static_cast<size_t>(pos) * half + i] = static_cast<float>(std::sin(angle));
+      }
+    }
+    base += static_cast<size_t>(extent[a]) * half;
+  }
+  return ROTA_OK;
+}
+
+rota_status rota_attn_prepare_qk(const rota_attn_desc* d, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                 const uint8_t* head_flags, const rota_attn_buffers* buf, void* stream) {
+  rota_status st = rota_attn_validate(d);
+  if (st != ROTA_OK) return st;
+  if (!buf || !q || !k || !v || !buf->rope_cos || !buf->rope_sin) return ROTA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return ROTA_ERR_INVALID_ARG;
+  int16_t tmp[256];
+  const int n_int4 = select_heads(d, head_flags, 0, tmp);
+  const int n_fp16 = d->H - n_int4;
+  if (n_int4 > 0) {
+    const void* need[] = {buf->q_codes, buf->k_codes, buf->q_scale, buf->k_scale, buf->v_codes, buf->v_scale};
+    for (const void* ptr : need)
+      if (!ptr || !aligned16(ptr)) return ROTA_ERR_INVALID_ARG;
+  }
+  if (n_fp16 > 0 && (!buf->q_rope || !buf->k_rope || !aligned16(buf->q_rope) || !aligned16(buf->k_rope)))
+    return ROTA_ERR_INVALID_ARG;
+
+  rota::PrologueParams p{};
+  p.q = reinterpret_cast<const __half*>(q);
+  p.k = reinterpret_cast<const __half*>(k);
+  p.v = reinterpret_cast<const __half*>(v);
+  p.q_codes = buf->q_codes;
+  p.k_codes = buf->k_codes;
+  p.q_scale = buf->q_scale;
+  p.k_scale = buf->k_scale;
+  p.v_codes = buf->v_codes;
+  p.v_scale = buf->v_scale;
+  p.q_rope = reinterpret_cast<__half*>(buf->q_rope);
+  p.k_rope = reinterpret_cast<__half*>(buf->k_rope);
+  p.cos_tab = buf->rope_cos;
+  p.sin_tab = buf->rope_sin;
+  p.H = d->H;
+  p.N = d->N;
+  p.nblk = npad_of(d->N) / 64;
+  p.grid_h = d->grid_h;
+  p.grid_w = d->grid_w;
+  const int extent[3] = {d->grid_t, d->grid_h, d->grid_w};
+  int coff = 0, toff = 0;
+  for (int a = 0; a < 3; ++a) {
+    p.rope_dim[a] = d->rope_dim[a];
+    p.had[a] = d->had_block[a];
+    p.unit[a] = d->had_block[a] < 2 ? 2 : d->had_block[a];
+    p.coff[a] = coff;
+    p.toff[a] = toff;
+    p.rnorm[a] = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d->had_block[a])));
+    coff += d->rope_dim[a];
+    toff += extent[a] * (d->rope_dim[a] / 2);
+  }
+  for (int h = 0; h < d->H; ++h)
+    if (head_flags && head_flags[h]) p.flags[h >> 5] |= 1u << (h & 31);
+
+  const dim3 grid(p.nblk, d->H, d->B * 3);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d->head_dim == 128)
+    rota::prologue_kernel<128><<<grid, rota::kPrologueThreads, 0, s>>>(p);
+  else
+    rota::prologue_kernel<64><<<grid, rota::kPrologueThreads, 0, s>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers* buf, const uint8_t* head_flags,
+                               float* out, void* stream, bool dump, int b, int h, int r0, int nr, int32_t* s_out,
+                               uint8_t* p_out) {
+  rota_status st = rota_attn_validate(d);
+  if (st != ROTA_OK) return st;
+  if (!buf || !out || !aligned16(out)) return ROTA_ERR_INVALID_ARG;
+  const void* need[] = {buf->q_codes, buf->k_codes, buf->q_scale, buf->k_scale, buf->v_codes, buf->v_scale};
+  for (const void* ptr : need)
+    if (!ptr || !aligned16(ptr)) return ROTA_ERR_INVALID_ARG;
+
+  static rota::Int4Params p;  // large (heads list); filled under a lock below
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  p = rota::Int4Params{};
+  p.q_codes = buf->q_codes;
+  p.k_codes = buf->k_codes;
+  p.q_scale = buf->q_scale;
+  p.k_scale = buf->k_scale;
+  p.v_codes = buf->v_codes;
+  p.v_scale = buf->v_scale;
+  p.out = out;
+  p.H = d->H;
+  p.N = d->N;
+  p.nblk = npad_of(d->N) / 64;
+  p.kappa = kappa_of(d);
+  std::memcpy(p.tau, tau_table().tau, sizeof(p.tau));
+  {
+    std::lock_guard<std::mutex> g(g_inject.mu);
+    p.timeout_ns = g_inject.armed ? g_inject.timeout_ns : kDefaultTimeoutNs;
+    p.inject_skip = g_inject.armed;
+    g_inject.armed = 0;
+  }
+  int batches = d->B;
+  if (dump) {
+    if (b < 0 || b >= d->B || h < 0 || h >= d->H || r0 < 0 || nr < 1 || r0 + nr > d->N || !s_out || !p_out)
+      return ROTA_ERR_INVALID_ARG;
+    p.nheads = 1;
+    p.heads[0] = static_cast<int16_t>(h);
+    p.s_dump = s_out;
+    p.p_dump = p_out;
+    p.dbg_r0 = r0;
+    p.dbg_nr = nr;
+    batches = 1;
+    // the kernel indexes batch by blockIdx.z; shift the base pointers to batch b
+    const size_t hs = static_cast<size_t>(b) * d->H;
+    const size_t npad = npad_of(d->N), nblk = npad / 64, D = d->head_dim;
+    p.q_codes += hs * npad * D / 2;
+    p.k_codes += hs * npad * D / 2;
+    p.q_scale += hs * nblk;
+    p.k_scale += hs * nblk;
+    p.v_codes += hs * nblk * D * 32;
+    p.v_scale += hs * nblk * D;
+    p.out += hs * d->N * D;
+  } else {
+    p.nheads = select_heads(d, head_flags, 0, p.heads);
+    if (p.nheads == 0) return ROTA_OK;
+  }
+  const dim3 grid((d->N + rota::kBM - 1) / rota::kBM, p.nheads, batches);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d->head_dim == 128) {
+    using L = rota::Int4Smem<128>;
+    if (dump) {
+      if ((st = set_smem(rota::attn_int4_kernel<128, true>, L::ALLOC)) != ROTA_OK) return st;
+      rota::attn_int4_kernel<128, true><<<grid, rota::kInt4Threads, L::ALLOC, s>>>(p);
+    } else {
+      if ((st = set_smem(rota::attn_int4_kernel<128, false>, L::ALLOC)) != ROTA_OK) return st;
+      rota::attn_int4_kernel<128, false><<<grid, rota::kInt4Threads, L::ALLOC, s>>>(p);
+    }
+  } else {
+    using L = rota::Int4Smem<64>;
+    if (dump) {
+      if ((st = set_smem(rota::attn_int4_kernel<64, true>, L::ALLOC)) != ROTA_OK) return st;
+      rota::attn_int4_kernel<64, true><<<grid, rota::kInt4Threads, L::ALLOC, s>>>(p);
+    } else {
+      if ((st = set_smem(rota::attn_int4_kernel<64, false>, L::ALLOC)) != ROTA_OK) return st;
+      rota::attn_int4_kernel<64, false><<<grid, rota::kInt4Threads, L::ALLOC, s>>>(p);
+    }
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+rota_status rota_attn_fwd_int4(const rota_attn_desc* d, const rota_attn_buffers* buf, const uint8_t* head_flags,
+                               float* out, void* stream) {
+  return launch_int4(d, buf, head_flags, out, stream, false, 0, 0, 0, 0, nullptr, nullptr);
+}
+
+rota_status rota_attn_debug_dump_int4(const rota_attn_desc* d, const rota_attn_buffers* buf, int32_t b, int32_t h,
+                                      int32_t r0, int32_t nr, int32_t* s_out, uint8_t* p_out, float* out,
+                                      void* stream) {
+  return launch_int4(d, buf, nullptr, out, stream, true, b, h, r0, nr, s_out, p_out);
+}
+
+rota_status rota_attn_fwd_fp16_fallback(const rota_attn_desc* d, const rota_attn_buffers* buf, const uint16_t* v,
+                                        const uint8_t* head_flags, float* out, void* stream) {
+  rota_status st = rota_attn_validate(d);
+  if (st != ROTA_OK) return st;
+  if (!buf || !v || !out || !aligned16(v) || !aligned16(out)) return ROTA_ERR_INVALID_ARG;
+  static rota::Fp16Params p;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  p = rota::Fp16Params{};
+  p.nheads = select_heads(d, head_flags, 1, p.heads);
+  if (p.nheads == 0) return ROTA_OK;
+  if (!buf->q_rope || !buf->k_rope || !aligned16(buf->q_rope) || !aligned16(buf->k_rope)) return ROTA_ERR_INVALID_ARG;
+  p.q_rope = reinterpret_cast<const __half*>(buf->q_rope);
+  p.k_rope = reinterpret_cast<const __half*>(buf->k_rope);
+  p.v = reinterpret_cast<const __half*>(v);
+  p.out = out;
+  p.H = d->H;
+  p.N = d->N;
+  p.scale_log2 = kappa_of(d);
+  p.timeout_ns = kDefaultTimeoutNs;
+  const dim3 grid((d->N + rota::kBM - 1) / rota::kBM, p.nheads, d->B);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d->head_dim == 128) {
+    using L = rota::F16Smem<128>;
+    if ((st = set_smem(rota::attn_fp16_kernel<128>, L::ALLOC)) != ROTA_OK) return st;
+    rota::attn_fp16_kernel<128><<<grid, rota::kF16Threads, L::ALLOC, s>>>(p);
+  } else {
+    using L = rota::F16Smem<64>;
+    if ((st = set_smem(rota::attn_fp16_kernel<64>, L::ALLOC)) != ROTA_OK) return st;
+    rota::attn_fp16_kernel<64><<<grid, rota::kF16Threads, L::ALLOC, s>>>(p);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+rota_status rota_attn_get_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_status(e);
+  int v = 0, zero = 0;
+  if ((e = cudaMemcpyFromSymbol(&v, rota::g_error, sizeof(int))) != cudaSuccess) return cuda_status(e);
+  if ((e = cudaMemcpyToSymbol(rota::g_error, &zero, sizeof(int))) != cudaSuccess) return cuda_status(e);
+  if (v == rota::kDevTimeout) return ROTA_ERR_TIMEOUT;
+  if (v != 0) return ROTA_ERR_DEVICE;
+  return ROTA_OK;
+}
+
+rota_status rota_attn_debug_pcode(const float* dvals, uint8_t* u, int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (!dvals || !u))) return ROTA_ERR_INVALID_ARG;
+  if (n == 0) return ROTA_OK;
+  rota::Int4Params p{};
+  std::memcpy(p.tau, tau_table().tau, sizeof(p.tau));
+  const int64_t blocks64 = (n + 255) / 256;
+  const int blocks = static_cast<int>(blocks64 < 148 * 16 ? blocks64 : 148 * 16);
+  rota::pcode_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(dvals, u, n, p);
+  return cuda_status(cudaGetLastError());
+}
+
+rota_status rota_attn_debug_inject_timeout(int32_t arm, uint64_t timeout_ns) {
+  std::lock_guard<std::mutex> g(g_inject.mu);
+  g_inject.armed = arm ? 1 : 0;
+  g_inject.timeout_ns = timeout_ns ? timeout_ns : kDefaultTimeoutNs;
+  return ROTA_OK;
+}
+
+}  // extern "C"
