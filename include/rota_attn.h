@@ -174,6 +174,36 @@ rota_status rota_attn_get_error(void* stream);
 /* Static string for a status code. */
 const char* rota_attn_status_string(rota_status s);
 
+/*
+ * Allocation-free INT4 forward (the paper has no counterpart: this is a
+ * packaging of rota_attn_prepare_qk + rota_attn_fwd_int4 for callers that
+ * cannot allocate device memory -- a plugin inside a host application that
+ * owns the device allocator, or a real-time loop where an allocation could
+ * synchronise the device or fail).  The caller passes only the inputs
+ * q, k, v (fp16 [B,H,N,head_dim]) and the output out (fp32 [B,H,N,head_dim]);
+ * every head takes the INT4 path (no FP16 fallback).  The intermediate codes,
+ * scales and RoPE tables live in one 16 MiB array in the library's static
+ * device memory, which every GPU that loads the library holds until exit.
+ * Its size bounds the problem: B*H*nblk*(96*head_dim + 4*head_dim + 8) bytes
+ * of codes and scales plus the RoPE tables (each entry padded to 256 bytes)
+ * must fit in ROTA_NOALLOC_SCRATCH_BYTES, and each RoPE table in
+ * ROTA_NOALLOC_MAX_TABLE floats; larger problems return
+ * ROTA_ERR_UNSUPPORTED, with nothing enqueued.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  The RoPE tables are copied from a static host
+ * buffer with a pageable cudaMemcpyAsync, which synchronises `stream` first.
+ * All calls share the one array and it keeps the last call's contents (every
+ * byte a call reads is written earlier in the same call, so nothing has to
+ * start at zero); calls whose device work overlaps -- on two streams, or from
+ * two host threads -- race on it.  No cudaMalloc, cudaFree or other
+ * allocating routine is called.
+ */
+#define ROTA_NOALLOC_SCRATCH_BYTES (16u << 20)
+#define ROTA_NOALLOC_MAX_TABLE (1u << 14)
+rota_status rota_attn_fwd_int4_noalloc(const rota_attn_desc* desc, const uint16_t* q, const uint16_t* k,
+                                       const uint16_t* v, float* out, void* stream);
+
 /* ---------------------------------------------------------- test hooks --- */
 
 /*

@@ -381,3 +381,86 @@ rota_status rota_attn_debug_inject_timeout(int32_t arm, uint64_t timeout_ns) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free INT4 forward: the codes, scales and RoPE tables of one call
+// live in a static device array instead of caller-allocated buffers.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[ROTA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+
+struct NoAllocState {
+  std::mutex mu;
+  void* scratch[kMaxDevices] = {};            // device address of g_noalloc_scratch, per device
+  float host_cos[ROTA_NOALLOC_MAX_TABLE];     // staging for the RoPE tables (no heap allocation)
+  float host_sin[ROTA_NOALLOC_MAX_TABLE];
+} g_noalloc;
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Set-up, once per device, with that device current: the symbol's device address.
+rota_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (dev < 0 || dev >= kMaxDevices) return ROTA_ERR_UNSUPPORTED;
+  if (!g_noalloc.scratch[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_status(e);
+    g_noalloc.scratch[dev] = p;
+  }
+  *out = g_noalloc.scratch[dev];
+  return ROTA_OK;
+}
+
+}  // namespace
+
+extern "C" rota_status rota_attn_fwd_int4_noalloc(const rota_attn_desc* d, const uint16_t* q, const uint16_t* k,
+                                                  const uint16_t* v, float* out, void* stream) {
+  rota_status st = rota_attn_validate(d);
+  if (st != ROTA_OK) return st;
+  if (!q || !k || !v || !out) return ROTA_ERR_INVALID_ARG;
+  size_t sz[ROTA_BUF_COUNT];
+  if ((st = rota_attn_buffer_sizes(d, sz)) != ROTA_OK) return st;
+  const size_t table_floats = sz[ROTA_BUF_ROPE_TABLE] / 4;
+  const int order[] = {ROTA_BUF_Q_CODES, ROTA_BUF_K_CODES, ROTA_BUF_Q_SCALE, ROTA_BUF_K_SCALE,
+                       ROTA_BUF_V_CODES, ROTA_BUF_V_SCALE, ROTA_BUF_ROPE_TABLE, ROTA_BUF_ROPE_TABLE};
+  size_t off[8], total = 0;
+  for (int i = 0; i < 8; ++i) {
+    off[i] = total;
+    total += round256(sz[order[i]]);
+  }
+  if (total > ROTA_NOALLOC_SCRATCH_BYTES || table_floats > ROTA_NOALLOC_MAX_TABLE) {
+    std::fprintf(stderr,
+                 "rota_attn_fwd_int4_noalloc: problem needs %zu bytes of scratch and %zu-entry RoPE tables; "
+                 "the static scratch holds %u bytes and %u entries\n",
+                 total, table_floats, ROTA_NOALLOC_SCRATCH_BYTES, ROTA_NOALLOC_MAX_TABLE);
+    return ROTA_ERR_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc.mu);
+  void* base = nullptr;
+  if ((st = noalloc_scratch(&base)) != ROTA_OK) return st;
+  uint8_t* s = static_cast<uint8_t*>(base);
+  if ((st = rota_attn_build_rope_tables(d, g_noalloc.host_cos, g_noalloc.host_sin)) != ROTA_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // Pageable source: returns once the host buffer has been consumed.
+  cudaError_t e = cudaMemcpyAsync(s + off[6], g_noalloc.host_cos, sz[ROTA_BUF_ROPE_TABLE], cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(s + off[7], g_noalloc.host_sin, sz[ROTA_BUF_ROPE_TABLE], cudaMemcpyHostToDevice, cs);
+  if (e != cudaSuccess) return cuda_status(e);
+  rota_attn_buffers b{};
+  b.q_codes = s + off[0];
+  b.k_codes = s + off[1];
+  b.q_scale = reinterpret_cast<float*>(s + off[2]);
+  b.k_scale = reinterpret_cast<float*>(s + off[3]);
+  b.v_codes = s + off[4];
+  b.v_scale = reinterpret_cast<float*>(s + off[5]);
+  b.rope_cos = reinterpret_cast<const float*>(s + off[6]);
+  b.rope_sin = reinterpret_cast<const float*>(s + off[7]);
+  if ((st = rota_attn_prepare_qk(d, q, k, v, nullptr, &b, stream)) != ROTA_OK) return st;
+  return rota_attn_fwd_int4(d, &b, nullptr, out, stream);
+}

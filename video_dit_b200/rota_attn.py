@@ -59,6 +59,7 @@ _SIGS = {
                                    ctypes.c_int32, _P, _P, _P, _P], ctypes.c_int),
     "rota_attn_debug_pcode": ([_P, _P, ctypes.c_int64, _P], ctypes.c_int),
     "rota_attn_debug_inject_timeout": ([ctypes.c_int32, ctypes.c_uint64], ctypes.c_int),
+    "rota_attn_fwd_int4_noalloc": ([_D, _P, _P, _P, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -135,6 +136,13 @@ def rota_attn_fwd_int4(desc, buffers: rota_attn_buffers, head_flags, out, stream
 def rota_attn_fwd_fp16_fallback(desc, buffers: rota_attn_buffers, v, head_flags, out, stream=None) -> int:
     return _lib.rota_attn_fwd_fp16_fallback(ctypes.byref(desc), ctypes.byref(buffers), _ptr(v),
                                             _flags(head_flags), _ptr(out), _stream(stream))
+
+
+def rota_attn_fwd_int4_noalloc(desc, q, k, v, out, stream=None) -> int:
+    """All-INT4 forward whose intermediates live in the library's static
+    device scratch (for callers that cannot allocate device memory)."""
+    return _lib.rota_attn_fwd_int4_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                           _stream(stream))
 
 
 def rota_attn_get_error(stream=None) -> int:
