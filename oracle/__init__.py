@@ -59,6 +59,10 @@ def lib():
         L.oracle_quant_params.restype = None
         L.oracle_quant_code.argtypes = [f32, f32]
         L.oracle_quant_code.restype = i32
+        L.oracle_pack_codes.argtypes = [P, i64, P]
+        L.oracle_pack_codes.restype = None
+        L.oracle_code_at.argtypes = [P, i64]
+        L.oracle_code_at.restype = i32
         L.oracle_quant_codes.argtypes = [P, i64, f32, P]
         L.oracle_quant_codes.restype = None
         L.oracle_prepare.argtypes = [i32, i32, i32, i32, P, P, P, f64] + [P] * 12
@@ -239,10 +243,22 @@ def attn_ref(q, k, v, grid, rope_dim, sm_scale: float, b: int, h: int, r0: int, 
     return out
 
 
-def unpack_s4(packed: np.ndarray) -> np.ndarray:
-    """Two's-complement nibbles (low nibble first) -> int8, last axis doubled."""
-    lo = (packed & 0xF).astype(np.int8)
-    hi = (packed >> 4).astype(np.int8)
-    lo = np.where(lo >= 8, lo - 16, lo).astype(np.int8)
-    hi = np.where(hi >= 8, hi - 16, hi).astype(np.int8)
-    return np.stack([lo, hi], axis=-1).reshape(*packed.shape[:-1], packed.shape[-1] * 2)
+def pack_codes(v: np.ndarray) -> np.ndarray:
+    """Codes in [-7, 7] (last axis a multiple of 8) -> the packed byte layout."""
+    v = np.ascontiguousarray(v, dtype=np.int32)
+    out = np.empty(v.shape[:-1] + (v.shape[-1] // 2,), np.uint8)
+    lib().oracle_pack_codes(_p(v), v.size, _p(out))
+    return out
+
+
+def unpack_codes(packed: np.ndarray) -> np.ndarray:
+    """Packed code bytes -> int8 codes (last axis doubled), via the oracle's reader."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    n = packed.shape[-1] * 2
+    flat = packed.reshape(-1, packed.shape[-1])
+    out = np.empty((flat.shape[0], n), np.int8)
+    L = lib()
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        out[r] = [L.oracle_code_at(_p(row), i) for i in range(n)]
+    return out.reshape(packed.shape[:-1] + (n,))

@@ -214,6 +214,27 @@ int oracle_quant_code(float y, float inv)
     return (int)r;
 }
 
+static uint8_t nibble(int v) { return (uint8_t)(v < 0 ? (8 | -v) : v); }
+
+/* Packs n (multiple of 8) codes into n/2 bytes in the layout above. */
+static void pack_codes(const int *v, long n, uint8_t *out)
+{
+    for (long g = 0; g < n; g += 8)
+        for (int j = 0; j < 4; ++j)
+            out[g / 2 + j] = (uint8_t)(nibble(v[g + j]) | (nibble(v[g + j + 4]) << 4));
+}
+
+/* Element i of a packed row. */
+static int code_at(const uint8_t *row, long i)
+{
+    uint8_t byte = row[(i / 8) * 4 + (i % 4)];
+    int nib = (i % 8) < 4 ? (byte & 0xf) : (byte >> 4);
+    return (nib & 8) ? -(nib & 7) : (nib & 7);
+}
+
+void oracle_pack_codes(const int *v, long n, uint8_t *out) { pack_codes(v, n, out); }
+int oracle_code_at(const uint8_t *row, long i) { return code_at(row, i); }
+
 void oracle_quant_codes(const float *y, long n, float inv, int8_t *codes)
 {
     for (long i = 0; i < n; ++i) codes[i] = (int8_t)oracle_quant_code(y[i], inv);
@@ -223,8 +244,11 @@ void oracle_quant_codes(const float *y, long n, float inv, int8_t *codes)
 /* The prologue for one attention call.                                     */
 /*   q, k, v        : fp16 bits [B,H,N,d]                                   */
 /*   flags          : [H], 1 = head takes the FP16 fallback                 */
-/* Outputs (layouts are the library's interface; codes two per byte, low   */
-/* nibble = even channel/token, two's complement s4):                      */
+/* Outputs (layouts are the library's interface):                         */
+/*   a code v in [-7, 7] is a sign-magnitude nibble (bit 3 = sign,          */
+/*   bits 0-2 = |v|; zero is 0000); along the packed axis every 8           */
+/*   consecutive elements e0..e7 form one little-endian 32-bit word whose   */
+/*   byte j (0..3) holds e_j in its low nibble and e_{j+4} in its high one. */
 /*   q_codes,k_codes: [B,H,Npad,d/2]   q_scale,k_scale : [B,H,Npad/64]      */
 /*   v_codes        : [B,H,Npad/64,d,32] (64 tokens of one channel)         */
 /*   v_scale        : [B,H,Npad/64,d]                                       */
@@ -248,7 +272,8 @@ int oracle_prepare(int B, int H, int N, int d, const int grid[3], const int rope
     float *sin_tab = (float *)malloc(sizeof(float) * (size_t)tlen);
     float *x = (float *)malloc(sizeof(float) * (size_t)d);
     float *blk = (float *)malloc(sizeof(float) * (size_t)QB * d);
-    if (!cos_tab || !sin_tab || !x || !blk) return -1;
+    int *codes = (int *)malloc(sizeof(int) * (size_t)(d > QB ? d : QB));
+    if (!cos_tab || !sin_tab || !x || !blk || !codes) return -1;
     oracle_rope_tables(grid, rope_dim, theta, cos_tab, sin_tab);
 
     for (int b = 0; b < B; ++b) {
@@ -289,14 +314,9 @@ int oracle_prepare(int B, int H, int N, int d, const int grid[3], const int rope
                     sdst[t][j] = scale;
                     for (int r = 0; r < QB; ++r) {
                         long n = (long)j * QB + r;
-                        for (int c = 0; c < d; c += 2) {
-                            int c0 = 0, c1 = 0;
-                            if (n < N) {
-                                c0 = oracle_quant_code(blk[(long)r * d + c], inv);
-                                c1 = oracle_quant_code(blk[(long)r * d + c + 1], inv);
-                            }
-                            cdst[t][n * (d / 2) + c / 2] = (uint8_t)((c0 & 0xf) | ((c1 & 0xf) << 4));
-                        }
+                        for (int c = 0; c < d; ++c)
+                            codes[c] = (n < N) ? oracle_quant_code(blk[(long)r * d + c], inv) : 0;
+                        pack_codes(codes, d, cdst[t] + n * (d / 2));
                     }
                 }
             }
@@ -316,17 +336,14 @@ int oracle_prepare(int B, int H, int N, int d, const int grid[3], const int rope
                     float scale, inv;
                     oracle_quant_params(amax, &scale, &inv);
                     vsc[(long)j * d + c] = scale;
-                    for (int r = 0; r < QB; r += 2) {
-                        long n = (long)j * QB + r;
-                        int c0 = (n < N) ? oracle_quant_code(vals[r], inv) : 0;
-                        int c1 = (n + 1 < N) ? oracle_quant_code(vals[r + 1], inv) : 0;
-                        vc[((long)j * d + c) * 32 + r / 2] = (uint8_t)((c0 & 0xf) | ((c1 & 0xf) << 4));
-                    }
+                    for (int r = 0; r < QB; ++r)
+                        codes[r] = ((long)j * QB + r < N) ? oracle_quant_code(vals[r], inv) : 0;
+                    pack_codes(codes, QB, vc + ((long)j * d + c) * 32);
                 }
             }
         }
     }
-    free(cos_tab); free(sin_tab); free(x); free(blk);
+    free(cos_tab); free(sin_tab); free(x); free(blk); free(codes);
     return 0;
 }
 
@@ -355,12 +372,6 @@ int oracle_pcode(float d, int *bad)
 void oracle_pcode_array(const float *d, uint8_t *u, long n, int *bad)
 {
     for (long i = 0; i < n; ++i) u[i] = (uint8_t)oracle_pcode(d[i], bad);
-}
-
-static inline int s4(uint8_t byte, int hi)
-{
-    int v = hi ? (byte >> 4) : (byte & 0xf);
-    return v >= 8 ? v - 16 : v;
 }
 
 /* ----------------------------------------------------------------------- */
@@ -411,11 +422,11 @@ int oracle_attn_int4(int B, int H, int N, int d, float sm_scale, int group,
     if (!S || !cs || !U || !mg || !qrow || !num) return -1;
 
     for (int i = r0; i < r0 + nr; ++i) {
-        for (int c = 0; c < d; ++c) qrow[c] = s4(qc[(long)i * (d / 2) + c / 2], c & 1);
+        for (int c = 0; c < d; ++c) qrow[c] = code_at(qc + (long)i * (d / 2), c);
         float sq = qs[i / QB];
         for (long kk = 0; kk < N; ++kk) {
             long acc = 0;
-            for (int c = 0; c < d; ++c) acc += (long)qrow[c] * s4(kc[kk * (d / 2) + c / 2], c & 1);
+            for (int c = 0; c < d; ++c) acc += (long)qrow[c] * code_at(kc + kk * (d / 2), c);
             if (acc > 49L * d || acc < -49L * d) bad++;
             S[kk] = (int32_t)acc;
             float t = sq * ks[kk / QB];
@@ -444,7 +455,7 @@ int oracle_attn_int4(int B, int H, int N, int d, float sm_scale, int group,
                 if (U[kk] == 0) continue;
                 long j = kk / QB, t = kk % QB;
                 for (int c = 0; c < d; ++c) {
-                    int vcode = s4(vc[(j * d + c) * 32 + t / 2], (int)(t & 1));
+                    int vcode = code_at(vc + (j * d + c) * 32, t);
                     num[c] += w * (double)vsc[j * d + c] * (double)vcode;
                 }
             }
@@ -458,7 +469,7 @@ int oracle_attn_int4(int B, int H, int N, int d, float sm_scale, int group,
                     den += (double)U[kk];
                     long j = kk / QB, t = kk % QB;
                     for (int c = 0; c < d; ++c) {
-                        int vcode = s4(vc[(j * d + c) * 32 + t / 2], (int)(t & 1));
+                        int vcode = code_at(vc + (j * d + c) * 32, t);
                         num[c] += (double)U[kk] * (double)vsc[j * d + c] * (double)vcode;
                     }
                 }

@@ -23,6 +23,9 @@ CASES = {
     "ragged_small": synth.scaled(synth.WORKLOADS["wan480"], "ragged", H=1, grid=(1, 3, 7)),     # N=21 < 64
 }
 
+# Many key blocks per CTA (74), so every pipeline stage and barrier phase wraps many times.
+LONG = synth.scaled(synth.WORKLOADS["wan480"], "wan_long", H=2, grid=(3, 30, 52))           # N=4680
+
 
 def _oracle(w, q, k, v, flags=None):
     return oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block, w.theta, flags)
@@ -115,3 +118,18 @@ def test_pcode_function_exhaustive_near_thresholds():
     u = torch.empty(d.size, dtype=torch.uint8, device="cuda")
     ra._check(ra.rota_attn_debug_pcode(dd, u), "pcode")
     assert np.array_equal(u.cpu().numpy(), oracle.pcode_array(d))
+
+
+def test_int4_long_sequence_sampled_rows():
+    w = LONG
+    q, k, v = synth.make_inputs(w)
+    h, r0, nr = 1, w.N - 200, 200          # the last two CTAs of the head, ragged tail included
+    _, out, (s, p, _) = run(w, q, k, v, dump=(0, h, r0, nr))
+    ref = _oracle(w, q, k, v)
+    o_ref, s_ref, p_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, r0, nr, dump=True)
+    assert np.array_equal(s, s_ref)
+    assert np.array_equal(p, p_ref)
+    e, rel, cos = row_stats(out[0, h, r0:r0 + nr], o_ref)
+    assert e <= TOL, (e, rel, cos)
+    o0 = oracle.attn_int4(ref, w.N, sm_scale(w), 0, 0, 0, 64)          # first rows of the other head
+    assert row_stats(out[0, 0, :64], o0)[0] <= TOL

@@ -17,6 +17,8 @@ import torch
 import oracle
 from video_dit_b200 import synth
 
+from codes import unpack
+
 
 # ------------------------------------------------------------ fp16 casts ---
 
@@ -180,6 +182,20 @@ def test_quantiser_zero_block():
     assert oracle.quant_code(0.0, 0.0) == 0
 
 
+def test_code_packing_layout():
+    rng = np.random.default_rng(5)
+    v = rng.integers(-7, 8, size=(37, 64)).astype(np.int32)
+    packed = oracle.pack_codes(v)
+    assert packed.shape == (37, 32)
+    assert np.array_equal(unpack(packed), v)
+    # spot values: e0 = -3, e4 = 5 -> byte 0 = 0x5B; zero stays 0000
+    w = np.zeros((1, 8), np.int32)
+    w[0, 0], w[0, 4], w[0, 7] = -3, 5, -7
+    assert list(oracle.pack_codes(w)[0]) == [0x5B, 0x00, 0x00, 0xF0]
+    assert [oracle.lib().oracle_code_at(oracle._p(oracle.pack_codes(w)[0].copy()), i) for i in range(8)] == \
+        [-3, 0, 0, 0, 5, 0, 0, -7]
+
+
 # --------------------------------------------------------------- P codes ---
 
 def _thresholds():
@@ -234,14 +250,14 @@ def test_prepare_codes_reconstruct_rotated_values():
     q, k, v = synth.make_inputs(w)
     p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block)
     for name, src in (("q", q), ("k", k)):
-        codes = oracle.unpack_s4(p[f"{name}_codes"][0, 1]).astype(np.float64)
+        codes = unpack(p[f"{name}_codes"][0, 1]).astype(np.float64)
         scale = np.repeat(p[f"{name}_scale"][0, 1], 64).astype(np.float64)
         for n in range(0, w.N, 37):
             y = oracle.rope_rotate_row(src[0, 1, n].astype(np.float32), n, w.grid, w.rope_dim, w.had_block)
             assert np.abs(codes[n] * scale[n] - y).max() <= scale[n] / 2 * (1 + 1e-6)
         for j in range(w.N // 64):
             assert np.abs(codes[j * 64:(j + 1) * 64]).max() == 7
-    vc = oracle.unpack_s4(p["v_codes"][0, 0]).astype(np.float64)       # [blk, d, 64]
+    vc = unpack(p["v_codes"][0, 0]).astype(np.float64)       # [blk, d, 64]
     vs = p["v_scale"][0, 0].astype(np.float64)                          # [blk, d]
     deq = (vc * vs[:, :, None]).transpose(0, 2, 1).reshape(-1, w.d)
     vv = v[0, 0].astype(np.float64)
@@ -253,8 +269,8 @@ def test_integer_scores_brute_force():
     q, k, v = synth.make_inputs(w)
     p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block)
     _, s, _ = oracle.attn_int4(p, w.N, 1 / math.sqrt(w.d), 0, 1, 0, w.N, dump=True)
-    qc = oracle.unpack_s4(p["q_codes"][0, 1]).astype(np.int64)
-    kc = oracle.unpack_s4(p["k_codes"][0, 1]).astype(np.int64)
+    qc = unpack(p["q_codes"][0, 1]).astype(np.int64)
+    kc = unpack(p["k_codes"][0, 1]).astype(np.int64)
     assert np.array_equal(s, qc @ kc.T)
 
 
@@ -266,7 +282,7 @@ def test_pcodes_span_full_range_and_offset_identity():
     for h in range(w.H):
         _, _, u = oracle.attn_int4(p, w.N, 1 / math.sqrt(w.d), 0, h, 0, w.N, dump=True)
         hist += np.bincount(u.ravel(), minlength=16)
-        vc = oracle.unpack_s4(p["v_codes"][0, h]).astype(np.int64)    # [blk, d, 64]
+        vc = unpack(p["v_codes"][0, h]).astype(np.int64)    # [blk, d, 64]
         for j in range(w.N // 64):
             uj = u[:, j * 64:(j + 1) * 64].astype(np.int64)
             lhs = uj @ vc[j].T
@@ -293,7 +309,7 @@ def test_uniform_attention_when_scores_vanish():
     p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block)
     out, _, u = oracle.attn_int4(p, w.N, 1 / math.sqrt(w.d), 0, 0, 0, w.N, dump=True)
     assert np.all(u == 15)
-    vc = oracle.unpack_s4(p["v_codes"][0, 0]).astype(np.float64)
+    vc = unpack(p["v_codes"][0, 0]).astype(np.float64)
     deq = (vc * p["v_scale"][0, 0].astype(np.float64)[:, :, None]).transpose(0, 2, 1).reshape(-1, w.d)
     assert np.abs(out - deq[: w.N].mean(axis=0)[None]).max() < 1e-12
 
@@ -309,7 +325,7 @@ def test_dominant_key_selects_its_value_row():
     p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block)
     out, s, u = oracle.attn_int4(p, w.N, 1 / math.sqrt(w.d), 0, 0, j, 1, dump=True)
     assert u[0, j] == 15 and u[0].sum() == 15
-    vc = oracle.unpack_s4(p["v_codes"][0, 0]).astype(np.float64)
+    vc = unpack(p["v_codes"][0, 0]).astype(np.float64)
     row = vc[j // 64, :, j % 64] * p["v_scale"][0, 0, j // 64].astype(np.float64)
     assert np.abs(out[0] - row).max() < 1e-12
 
@@ -329,7 +345,7 @@ def test_single_group_is_global_max():
     M = x.max(axis=1, keepdims=True)
     dd = (s.astype(np.float64) * c.astype(np.float64) - M).astype(np.float32)  # one rounding
     assert np.array_equal(u, oracle.pcode_array(dd))
-    vc = oracle.unpack_s4(p["v_codes"][0, 0]).astype(np.float64)
+    vc = unpack(p["v_codes"][0, 0]).astype(np.float64)
     deq = (vc * p["v_scale"][0, 0].astype(np.float64)[:, :, None]).transpose(0, 2, 1).reshape(-1, w.d)
     want = (u.astype(np.float64) @ deq[: w.N]) / u.sum(axis=1, keepdims=True)
     assert np.abs(out - want).max() < 1e-12

@@ -6,17 +6,28 @@
 // fixed scale and zero-point so that all 16 unsigned 4-bit levels are used
 // ("Range-optimized P Quantization").
 //
-// Per CTA: 128 query rows of one head; thread i owns row i (TMEM lane i).
-// Per 64-key block:
-//   1. packed s4 K / V codes -> s8 in shared memory (128-bit loads, swizzled
-//      K-major layouts the tensor core reads directly);
-//   2. S = Qc Kc^T on the tensor core (tcgen05.mma kind::i8, s32 in TMEM);
-//   3. per row: c = RN(RN(sq sk) kappa), running max m over the block,
-//      d = fma(S, c, -m), u = rne(15 * 2^d) (exact: estimate + threshold fix),
-//      row sum l and the u8 codes written to shared memory;
-//   4. acc = P V_c on the tensor core (kind::i8, u8 x s8 -> s32 in TMEM);
-//   5. O = O * 2^(m_old - m) + v_scale * acc in fp32 registers.
-// The epilogue writes O / l.
+// Exact integer contractions on the 8-bit tensor-core path.  A code v in
+// [-7, 7] is widened to the e4m3 subnormal v * 2^-9 (exact), a P code u in
+// 0..15 to the e4m3 normal u (exact), and tcgen05.mma kind::f8f6f4 sums the
+// products in fp32: every partial sum is an integer multiple of 2^-18 (S) or
+// 2^-9 (P V) far below 2^24 units, so S = S_int * 2^-18 and acc = acc_int *
+// 2^-9 hold exactly -- the same integers an s32 accumulation gives, already
+// in fp32 for the softmax and the V scales.
+//
+// One CTA = two 128-row query tiles of one head (256 rows), 384 threads:
+//   warp 0      TMA producer: packed K / V codes and V scales of each 64-key
+//               block -> a 4-slot shared-memory staging ring (cp.async.bulk);
+//   warp 1      TMEM owner and MMA issuer (one thread);
+//   warps 2-3   widen the staged nibbles into the swizzled K-major e4m3 K and
+//               V^T operand tiles (3 stages) -- once per block for both tiles;
+//   warps 4-7   query tile 0, warps 8-11 query tile 1 (thread = row = TMEM lane):
+//               running max, P codes, O update, epilogue.
+// Per 64-key block j and tile t the MMA warp issues S_t = Q_t K_j^T (128 x 64)
+// and, once tile t has written its P codes, PV_t = P_t [V_j^T; 1] (128 x (D+16));
+// the 16 extra columns of ones return the row sum of the P codes.  The two
+// tiles alternate, so the tensor core works on one while the other's CUDA
+// cores run the softmax; each tile's S buffer is released as soon as its
+// warps have loaded it, so S_t(j+1) overlaps the softmax of block j.
 #pragma once
 #include <climits>
 #include <cstdint>
@@ -46,264 +57,473 @@ struct Int4Params {
   int dbg_r0, dbg_nr;
 };
 
-constexpr int kInt4Threads = 128;
+constexpr int kInt4Threads = 384;
+constexpr int kRowsPerCta = 2 * kBM;
+constexpr int kStg = 4;   // staging slots
+constexpr int kOps = 3;   // widened operand stages
+constexpr int kProducerRegs = 40;
+constexpr int kConsumerRegs = 232;
+// Register split: kProducerRegs * 128 + kConsumerRegs * 256 equals the launch
+// allocation 384 * kLaunchRegs; the host refuses to launch a build whose
+// register count differs (setmaxnreg.inc would otherwise wait forever).
+constexpr int kLaunchRegs = (kProducerRegs * 128 + kConsumerRegs * 256) / 384;
+static_assert(kLaunchRegs * 384 == kProducerRegs * 128 + kConsumerRegs * 256, "register split");
 
 template <int D>
 struct Int4Smem {
-  static constexpr int QROW = D;          // bytes per s8 row of Q / K
-  static constexpr int Q_BYTES = kBM * D;
-  static constexpr int K_BYTES = kBN * D;
-  static constexpr int V_BYTES = D * kBN;  // V^T: D rows of 64 keys
-  static constexpr int P_BYTES = kBM * kBN;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + K_BYTES;
-  static constexpr int OFF_P = OFF_V + V_BYTES;
-  static constexpr int OFF_VS = OFF_P + P_BYTES;       // D floats
-  static constexpr int OFF_TAU = OFF_VS + D * 4;       // 16 floats
-  static constexpr int OFF_BAR = OFF_TAU + 64;         // 8-byte aligned
-  static constexpr int OFF_TMEM = OFF_BAR + 8;
-  static constexpr int OFF_FLAG = OFF_TMEM + 4;
-  static constexpr int BYTES = OFF_FLAG + 4;
-  static constexpr int ALLOC = BYTES + 1024;           // + alignment slack
-  static constexpr int TMEM_COLS = (kBN + D) <= 128 ? 128 : 256;
+  static constexpr int NPV = D + 16;          // P V columns: D channels + 16 ones (row sum)
+  static constexpr int ROWB = D;              // bytes per e4m3 Q / K row
   static constexpr uint32_t LAYOUT_QK = D == 128 ? 2u : 4u;  // 128B / 64B swizzle
   static constexpr uint32_t SBO_QK = 8 * D;
+  static constexpr int KPACK = kBN * D / 2;
+  static constexpr int VPACK = D * kBN / 2;
+  static constexpr int STG_BYTES = KPACK + VPACK + D * 4;
+  static constexpr int Q_BYTES = kBM * D;
+  static constexpr int K_BYTES = kBN * D;
+  static constexpr int V_BYTES = ((NPV * kBN + 1023) / 1024) * 1024;
+  static constexpr int OP_BYTES = K_BYTES + V_BYTES;
+  static constexpr int P_BYTES = kBM * kBN;
+  static constexpr int OFF_Q = 0;                              // 2 tiles
+  static constexpr int OFF_OP = OFF_Q + 2 * Q_BYTES;           // kOps stages
+  static constexpr int OFF_P = OFF_OP + kOps * OP_BYTES;       // 2 tiles x 2 buffers
+  static constexpr int OFF_STG = OFF_P + 4 * P_BYTES;          // kStg slots
+  static constexpr int OFF_SV = OFF_STG + kStg * STG_BYTES;    // kOps x D floats: 512 * v_scale
+  static constexpr int OFF_TAU = OFF_SV + kOps * D * 4;
+  static constexpr int OFF_BAR = OFF_TAU + 64;
+  // barriers: stg_full[4] stg_empty[4] op_full[3] op_empty[3] s_full[2] s_empty[2]
+  //           pv_full[2] pv_empty[2] q_full mma_done p_full[2 tiles][2 buffers]
+  static constexpr int NBAR = 4 + 4 + 3 + 3 + 2 + 2 + 2 + 2 + 1 + 1 + 4;
+  static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_ABORT = OFF_TMEM + 4;
+  static constexpr int BYTES = OFF_ABORT + 4;
+  static constexpr int ALLOC = BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_S0 = 0, T_S1 = kBN, T_PV0 = 2 * kBN, T_PV1 = 2 * kBN + NPV;
+  static_assert(T_PV1 + NPV <= TMEM_COLS, "TMEM budget");
+  static_assert(STG_BYTES % 16 == 0 && KPACK % 16 == 0 && VPACK % 16 == 0, "bulk copy sizes");
+  static_assert(OFF_OP % 1024 == 0 && OP_BYTES % 1024 == 0 && K_BYTES % 1024 == 0 && OFF_P % 1024 == 0,
+                "swizzle atom alignment");
+  static_assert(OFF_STG % 16 == 0 && STG_BYTES % 16 == 0 && OFF_BAR % 8 == 0, "alignment");
 };
 
-// Range-optimised P code u = rne(15 * 2^d) in exact arithmetic, d <= ~0.
+// Range-optimised P code u = rne(15 * 2^d) in exact arithmetic (d <= ~0).
 // The MUFU estimate is within ~4e-6 of 15 * 2^d; only when it falls within
 // 1e-4 of a half-integer is the decision taken by the exact threshold table.
-__device__ __forceinline__ uint32_t pcode(float d, const float* tau) {
+__device__ __forceinline__ float pcode_f(float d, const float* tau) {
   const float e = 15.f * ex2_approx(d);
-  const float r = __fsub_rn(__fadd_rn(e, 12582912.f), 12582912.f);  // rne to integer
+  float r = __fsub_rn(__fadd_rn(e, 12582912.f), 12582912.f);  // rne to integer
   const float fr = e - r;
-  uint32_t u = static_cast<uint32_t>(r);
   if (fabsf(fr) > 0.5f - 1e-4f) {
     int j = fr > 0.f ? static_cast<int>(r) + 1 : static_cast<int>(r);
     j = max(1, min(15, j));
-    u = d >= tau[j] ? j : j - 1;
+    r = static_cast<float>(d >= tau[j] ? j : j - 1);
   }
-  return u;
+  return r;
 }
+
+__device__ __forceinline__ uint32_t pcode(float d, const float* tau) {
+  return static_cast<uint32_t>(pcode_f(d, tau));
+}
+
+// Four P codes (exact integers 0..15 in fp32) -> four e4m3 bytes, u0 lowest.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float u0, float u1, float u2, float u3) {
+  uint32_t w;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(w)
+      : "f"(u0), "f"(u1), "f"(u2), "f"(u3));
+  return w;
+}
+
+__device__ __forceinline__ void setmaxnreg_producer() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory");
+}
+__device__ __forceinline__ void setmaxnreg_consumer() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 232;" ::: "memory");
+}
+static_assert(kProducerRegs == 40 && kConsumerRegs == 232, "setmaxnreg immediates");
 
 template <int D, bool DUMP>
 __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid_constant__ Int4Params p) {
   using L = Int4Smem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem + L::OFF_Q;
-  uint8_t* sK = smem + L::OFF_K;
-  uint8_t* sV = smem + L::OFF_V;
-  uint8_t* sP = smem + L::OFF_P;
-  float* sVs = reinterpret_cast<float*>(smem + L::OFF_VS);
-  float* sTau = reinterpret_cast<float*>(smem + L::OFF_TAU);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* stg_full = bars;
+  uint64_t* stg_empty = bars + 4;
+  uint64_t* op_full = bars + 8;
+  uint64_t* op_empty = bars + 11;
+  uint64_t* s_full = bars + 14;
+  uint64_t* s_empty = bars + 16;
+  uint64_t* pv_full = bars + 18;
+  uint64_t* pv_empty = bars + 20;
+  uint64_t* q_full = bars + 22;
+  uint64_t* mma_done = bars + 23;
+  // One barrier per P buffer (tile t, block parity): tile t may write P(j+1)
+  // before the MMA warp has waited for P(j), so a single barrier per tile
+  // could complete two phases ahead of its waiter.
+  uint64_t* p_full = bars + 24;  // p_full[2 * t + (j & 1)], phase (j >> 1) & 1
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
-  int* sAbort = reinterpret_cast<int*>(smem + L::OFF_FLAG);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(smem + L::OFF_ABORT);
+  float* sTau = reinterpret_cast<float*>(smem + L::OFF_TAU);
+  float* sSv = reinterpret_cast<float*>(smem + L::OFF_SV);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int qt = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = p.heads[blockIdx.y];
   const int b = blockIdx.z;
   const size_t head = (size_t)b * p.H + h;
   const int npad = p.nblk * kBN;
-  const int row = qt * kBM + tid;
+  const int nkb = p.nblk;
+  const uint64_t lim = p.timeout_ns;
 
   if (tid < 16) sTau[tid] = p.tau[tid];
   if (tid == 0) {
-    mbar_init(bar, 1);
-    fence_mbar_init();
+    for (int i = 0; i < kStg; ++i) {
+      mbar_init(&stg_full[i], 1);
+      mbar_init(&stg_empty[i], 2);
+    }
+    for (int i = 0; i < kOps; ++i) {
+      mbar_init(&op_full[i], 2);
+      mbar_init(&op_empty[i], 1 + 8);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&s_empty[t], 4);
+      mbar_init(&p_full[2 * t], 4);
+      mbar_init(&p_full[2 * t + 1], 4);
+      mbar_init(&pv_full[t], 1);
+      mbar_init(&pv_empty[t], 4);
+    }
+    mbar_init(q_full, 8);
+    mbar_init(mma_done, 1);
     *sAbort = 0;
+    fence_mbar_init();
   }
   __syncwarp();
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(sTmem, L::TMEM_COLS);
     tmem_relinquish();
   }
-
-  // Q tile: packed s4 rows -> s8, swizzled K-major.
-  {
-    const uint8_t* qsrc = p.q_codes + (head * npad + (size_t)qt * kBM) * (D / 2);
-    for (int i = tid; i < kBM * D / 32; i += kInt4Threads) {
-      const int r = i / (D / 32), c = i % (D / 32);
-      uint4 w = make_uint4(0, 0, 0, 0);
-      if (qt * kBM + r < npad) w = __ldg(reinterpret_cast<const uint4*>(qsrc + (size_t)r * (D / 2) + c * 16));
-      uint32_t o[8];
-      s4x8_to_s8(w.x, o[0], o[1]);
-      s4x8_to_s8(w.y, o[2], o[3]);
-      s4x8_to_s8(w.z, o[4], o[5]);
-      s4x8_to_s8(w.w, o[6], o[7]);
-      *reinterpret_cast<uint4*>(sQ + swz<L::QROW>(r, c * 32)) = make_uint4(o[0], o[1], o[2], o[3]);
-      *reinterpret_cast<uint4*>(sQ + swz<L::QROW>(r, c * 32 + 16)) = make_uint4(o[4], o[5], o[6], o[7]);
-    }
-  }
-  const float sq = row < npad ? __ldg(p.q_scale + head * p.nblk + row / kBN) : 0.f;
-
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sTmem;
-  const uint32_t t_lane = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t tS = tmem;        // columns [0, 64): S (s32)
-  const uint32_t tO = tmem + kBN;  // columns [64, 64 + D): P V accumulator (s32)
 
-  constexpr uint32_t ID_S = idesc(2, 1, 1, kBM, kBN);   // s8 x s8 -> s32, 128 x 64
-  constexpr uint32_t ID_PV = idesc(2, 0, 1, kBM, D);    // u8 x s8 -> s32, 128 x D
-
-  float O[D];
+  if (warp < 4) {
+    // ===================================================== producer warpgroup
+    setmaxnreg_producer();
+    if (warp == 0) {
+      if (lane == 0) {
+        // ---- TMA producer ----
+        int issued = 0;
+        for (int j = 0; j < nkb; ++j) {
+          const int slot = j % kStg;
+          if (!mbar_wait(&stg_empty[slot], ((j / kStg) & 1) ^ 1, lim)) { *sAbort = 1; break; }
+          if (*sAbort) break;
+          uint8_t* dst = smem + L::OFF_STG + slot * L::STG_BYTES;
+          mbar_arrive_expect_tx(&stg_full[slot], L::STG_BYTES);
+          bulk_g2s(dst, p.k_codes + (head * npad + (size_t)j * kBN) * (D / 2), L::KPACK, &stg_full[slot]);
+          bulk_g2s(dst + L::KPACK, p.v_codes + (head * p.nblk + j) * (size_t)D * 32, L::VPACK, &stg_full[slot]);
+          bulk_g2s(dst + L::KPACK + L::VPACK, p.v_scale + (head * p.nblk + j) * D, D * 4, &stg_full[slot]);
+          issued = j + 1;
+        }
+        // drain: every issued copy has landed before the CTA may exit
+        for (int j = (issued > kStg ? issued - kStg : 0); j < issued; ++j)
+          mbar_wait(&stg_full[j % kStg], (j / kStg) & 1, lim);
+      }
+    } else if (warp == 1) {
+      if (lane == 0) {
+        // ---- MMA issuer ----
+        constexpr uint32_t ID_S = idesc(1, 0, 0, kBM, kBN);      // e4m3 x e4m3 -> f32, 128 x 64
+        constexpr uint32_t ID_PV = idesc(1, 0, 0, kBM, L::NPV);  // 128 x (D + 16)
+        const uint32_t qa0 = smem_u32(smem + L::OFF_Q), qa1 = qa0 + L::Q_BYTES;
+        const uint32_t pbase = smem_u32(smem + L::OFF_P);  // P buffer (tile t, block j) at (2t + (j & 1)) * P_BYTES
+        bool ok = mbar_wait(q_full, 0, lim);
+        auto issue_s = [&](int j, int t) -> bool {
+          const int op = j % kOps;
+          if (!mbar_wait(&s_empty[t], (j & 1) ^ 1, lim)) return false;
+          tc_fence_after();
+          if (p.inject_skip && j == 0 && t == 0) return true;  // fault injection: never committed
+          const uint32_t ka = smem_u32(smem + L::OFF_OP + op * L::OP_BYTES);
+          const uint32_t qa = t ? qa1 : qa0;
 #pragma unroll
-  for (int c = 0; c < D; ++c) O[c] = 0.f;
-  float m = -INFINITY, l = 0.f;
-  uint32_t phase = 0;
-  bool aborted = false;
-
-#pragma unroll 1
-  for (int kb = 0; kb < p.nblk; ++kb) {
-    // ---- stage K and V codes of this block ----
-    const uint8_t* ksrc = p.k_codes + (head * npad + (size_t)kb * kBN) * (D / 2);
-    for (int i = tid; i < kBN * D / 32; i += kInt4Threads) {
-      const int r = i / (D / 32), c = i % (D / 32);
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(ksrc + (size_t)r * (D / 2) + c * 16));
-      uint32_t o[8];
-      s4x8_to_s8(w.x, o[0], o[1]);
-      s4x8_to_s8(w.y, o[2], o[3]);
-      s4x8_to_s8(w.z, o[4], o[5]);
-      s4x8_to_s8(w.w, o[6], o[7]);
-      *reinterpret_cast<uint4*>(sK + swz<L::QROW>(r, c * 32)) = make_uint4(o[0], o[1], o[2], o[3]);
-      *reinterpret_cast<uint4*>(sK + swz<L::QROW>(r, c * 32 + 16)) = make_uint4(o[4], o[5], o[6], o[7]);
-    }
-    const uint8_t* vsrc = p.v_codes + (head * p.nblk + kb) * (size_t)D * 32;
-    for (int i = tid; i < D * 2; i += kInt4Threads) {
-      const int c = i >> 1, hlf = i & 1;
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(vsrc + (size_t)c * 32 + hlf * 16));
-      uint32_t o[8];
-      s4x8_to_s8(w.x, o[0], o[1]);
-      s4x8_to_s8(w.y, o[2], o[3]);
-      s4x8_to_s8(w.z, o[4], o[5]);
-      s4x8_to_s8(w.w, o[6], o[7]);
-      *reinterpret_cast<uint4*>(sV + swz<64>(c, hlf * 32)) = make_uint4(o[0], o[1], o[2], o[3]);
-      *reinterpret_cast<uint4*>(sV + swz<64>(c, hlf * 32 + 16)) = make_uint4(o[4], o[5], o[6], o[7]);
-    }
-    if (tid < D) sVs[tid] = __ldg(p.v_scale + (head * p.nblk + kb) * D + tid);
-    const float sk = __ldg(p.k_scale + head * p.nblk + kb);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- S = Qc Kc^T ----
-    if (tid == 0) {
-      tc_fence_after();
-      if (!(p.inject_skip && kb == 0)) {
-        const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK);
+          for (int k = 0; k < D / 32; ++k)
+            mma_f8f6f4(tmem + (t ? L::T_S1 : L::T_S0), sdesc(qa + 32 * k, L::SBO_QK, L::LAYOUT_QK),
+                       sdesc(ka + 32 * k, L::SBO_QK, L::LAYOUT_QK), ID_S, k > 0);
+          mma_commit(&s_full[t]);
+          return true;
+        };
+        auto issue_pv = [&](int j) -> bool {
+          const int op = j % kOps;
+          const uint32_t va = smem_u32(smem + L::OFF_OP + op * L::OP_BYTES + L::K_BYTES);
+          for (int t = 0; t < 2; ++t) {
+            if (!mbar_wait(&p_full[2 * t + (j & 1)], (j >> 1) & 1, lim)) return false;
+            if (!mbar_wait(&pv_empty[t], (j & 1) ^ 1, lim)) return false;
+            tc_fence_after();
+            const uint32_t pa = pbase + (2 * t + (j & 1)) * L::P_BYTES;
 #pragma unroll
-        for (int k = 0; k < D / 32; ++k)
-          mma_i8(tS, sdesc(qa + 32 * k, L::SBO_QK, L::LAYOUT_QK), sdesc(ka + 32 * k, L::SBO_QK, L::LAYOUT_QK),
-                 ID_S, k > 0);
-        mma_commit(bar);
+            for (int k = 0; k < kBN / 32; ++k)
+              mma_f8f6f4(tmem + (t ? L::T_PV1 : L::T_PV0), sdesc(pa + 32 * k, 512, 4), sdesc(va + 32 * k, 512, 4),
+                         ID_PV, k > 0);
+            mma_commit(&pv_full[t]);
+          }
+          mma_commit(&op_empty[op]);
+          return true;
+        };
+        for (int j = 0; ok && j < nkb; ++j) {
+          if (!mbar_wait(&op_full[j % kOps], (j / kOps) & 1, lim)) { ok = false; break; }
+          tc_fence_after();
+          if (!issue_s(j, 0) || !issue_s(j, 1)) { ok = false; break; }
+          if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+          if (*sAbort) { ok = false; break; }
+        }
+        if (ok) ok = issue_pv(nkb - 1);
+        if (!ok) *sAbort = 1;
+        // every issued MMA completes before TMEM is released
+        mma_commit(mma_done);
+        mbar_wait(mma_done, 0, lim);
+      }
+    } else {
+      // ---- widening warps (2, 3): staged nibbles -> e4m3 operand tiles ----
+      const int wt = tid - 64;  // 0..63
+      // the constant ones rows D..D+15 of every V^T stage (e4m3 1.0 = 0x38)
+      for (int op = 0; op < kOps; ++op) {
+        uint8_t* vt = smem + L::OFF_OP + op * L::OP_BYTES + L::K_BYTES;
+        for (int i = wt; i < 16 * kBN / 16; i += 64)
+          *reinterpret_cast<uint4*>(vt + D * kBN + 16 * i) =
+              make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
+      }
+      for (int j = 0; j < nkb; ++j) {
+        const int slot = j % kStg, op = j % kOps;
+        if (!warp_wait(&stg_full[slot], (j / kStg) & 1, lim)) { *sAbort = 1; break; }
+        if (!warp_wait(&op_empty[op], ((j / kOps) & 1) ^ 1, lim)) { *sAbort = 1; break; }
+        if (warp_flag(sAbort)) break;
+        const uint8_t* sg = smem + L::OFF_STG + slot * L::STG_BYTES;
+        uint8_t* kt = smem + L::OFF_OP + op * L::OP_BYTES;
+        uint8_t* vt = kt + L::K_BYTES;
+        // K: 64 rows x D/2 bytes packed; a 16-byte chunk = 32 channels of one row
+        for (int i = wt; i < kBN * D / 32; i += 64) {
+          const int rr = i / (D / 32), cg = i % (D / 32);
+          const uint4 w = *reinterpret_cast<const uint4*>(sg + 16 * i);
+          uint32_t o[8];
+          codes8_to_e4m3(w.x, o[0], o[1]);
+          codes8_to_e4m3(w.y, o[2], o[3]);
+          codes8_to_e4m3(w.z, o[4], o[5]);
+          codes8_to_e4m3(w.w, o[6], o[7]);
+          *reinterpret_cast<uint4*>(kt + swz<L::ROWB>(rr, cg * 32)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(kt + swz<L::ROWB>(rr, cg * 32 + 16)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        // V: D channel rows x 32 bytes packed (64 keys); a chunk = 32 keys of one channel
+        for (int i = wt; i < D * 2; i += 64) {
+          const int c = i >> 1, hl = i & 1;
+          const uint4 w = *reinterpret_cast<const uint4*>(sg + L::KPACK + 16 * i);
+          uint32_t o[8];
+          codes8_to_e4m3(w.x, o[0], o[1]);
+          codes8_to_e4m3(w.y, o[2], o[3]);
+          codes8_to_e4m3(w.z, o[4], o[5]);
+          codes8_to_e4m3(w.w, o[6], o[7]);
+          *reinterpret_cast<uint4*>(vt + swz<64>(c, hl * 32)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(vt + swz<64>(c, hl * 32 + 16)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        // V scales x 2^9 (the weight of an e4m3-subnormal V code), exact
+        const float* vs = reinterpret_cast<const float*>(sg + L::KPACK + L::VPACK);
+        for (int c = wt; c < D; c += 64) sSv[op * D + c] = vs[c] * 512.f;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&op_full[op]);
+          mbar_arrive(&stg_empty[slot]);
+        }
       }
     }
-    if (!mbar_wait(bar, phase, p.timeout_ns)) *sAbort = 1;
-    phase ^= 1;
-    __syncthreads();
-    if (*sAbort) { aborted = true; break; }
-    tc_fence_after();
+  } else {
+    // ===================================================== query-tile warpgroups
+    setmaxnreg_consumer();
+    const int t = (warp - 4) >> 2;            // tile 0 or 1
+    const int r = tid & 127;                  // row within the tile = TMEM lane
+    const int row = blockIdx.x * kRowsPerCta + t * kBM + r;
+    const uint32_t t_lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + (t ? L::T_S1 : L::T_S0) + t_lane;
+    const uint32_t tPV = tmem + (t ? L::T_PV1 : L::T_PV0) + t_lane;
+    uint8_t* sQ = smem + L::OFF_Q + t * L::Q_BYTES;
+    uint8_t* sP0 = smem + L::OFF_P + 2 * t * L::P_BYTES;   // P buffers of this tile (block parity)
 
-    int32_t S[kBN];
+    // own Q row: packed codes -> e4m3 subnormals in the swizzled Q tile
     {
-      uint32_t r0[32], r1[32];
-      tmem_ld32(tS + t_lane, r0);
-      tmem_ld32(tS + t_lane + 32, r1);
-      tmem_ld_wait();
+      const uint8_t* qsrc = p.q_codes + (head * npad + (size_t)row) * (D / 2);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        S[j] = static_cast<int32_t>(r0[j]);
-        S[32 + j] = static_cast<int32_t>(r1[j]);
+      for (int cg = 0; cg < D / 32; ++cg) {
+        uint4 w = make_uint4(0, 0, 0, 0);
+        if (row < npad) w = __ldg(reinterpret_cast<const uint4*>(qsrc + cg * 16));
+        uint32_t o[8];
+        codes8_to_e4m3(w.x, o[0], o[1]);
+        codes8_to_e4m3(w.y, o[2], o[3]);
+        codes8_to_e4m3(w.z, o[4], o[5]);
+        codes8_to_e4m3(w.w, o[6], o[7]);
+        *reinterpret_cast<uint4*>(sQ + swz<L::ROWB>(r, cg * 32)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(sQ + swz<L::ROWB>(r, cg * 32 + 16)) = make_uint4(o[4], o[5], o[6], o[7]);
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_full);
     }
+    const float sq = row < npad ? __ldg(p.q_scale + head * p.nblk + row / kBN) : 0.f;
+    const float* ksc = p.k_scale + head * p.nblk;
 
-    // ---- running max, P codes, row sum ----
-    const int nvalid = min(kBN, p.N - kb * kBN);
-    const float c = __fmul_rn(__fmul_rn(sq, sk), p.kappa);
-    int smax = INT_MIN;
+    float O[D];
 #pragma unroll
-    for (int j = 0; j < kBN; ++j)
-      if (j < nvalid) smax = max(smax, S[j]);
-    const float m_new = fmaxf(m, __fmul_rn(static_cast<float>(smax), c));
-    const float alpha = ex2_approx(m - m_new);  // m = -inf on the first block: alpha = 0
-    m = m_new;
-    uint32_t usum = 0;
-    uint32_t pw[kBN / 4];
-#pragma unroll
-    for (int j4 = 0; j4 < kBN / 4; ++j4) {
-      uint32_t w = 0;
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const int j = 4 * j4 + t;
-        const float dd = __fmaf_rn(static_cast<float>(S[j]), c, -m);
-        uint32_t u = pcode(dd, sTau);
-        if (j >= nvalid) u = 0;
-        usum += u;
-        w |= u << (8 * t);
-      }
-      pw[j4] = w;
-    }
-    l = __fmaf_rn(l, alpha, static_cast<float>(usum));
-#pragma unroll
-    for (int j = 0; j < kBN / 16; ++j)
-      *reinterpret_cast<uint4*>(sP + swz<64>(tid, 16 * j)) = make_uint4(pw[4 * j], pw[4 * j + 1], pw[4 * j + 2], pw[4 * j + 3]);
-    if (DUMP && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr) {
-      const size_t base = (size_t)(row - p.dbg_r0) * p.N + (size_t)kb * kBN;
-      for (int j = 0; j < nvalid; ++j) {
-        p.s_dump[base + j] = S[j];
-        p.p_dump[base + j] = static_cast<uint8_t>((pw[j >> 2] >> (8 * (j & 3))) & 0xFF);
-      }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
+    for (int c = 0; c < D; ++c) O[c] = 0.f;
+    float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
+    bool aborted = false;
 
-    // ---- acc = P Vc ----
-    if (tid == 0) {
+    // O update of block i: O = O * alpha_i + (512 v_scale_i) * acc_i; the ones
+    // columns carry the sum of the block's P codes for l.
+    auto o_update = [&](int i, float alpha) -> bool {
+      if (!warp_wait(&pv_full[t], i & 1, lim)) return false;
+      // the V scales of block i were written by the widening warps before op_full
+      if (!warp_wait(&op_full[i % kOps], (i / kOps) & 1, lim)) return false;
       tc_fence_after();
-      const uint32_t pa = smem_u32(sP), va = smem_u32(sV);
+      const float* sv = sSv + (i % kOps) * D;
+      // alpha == 1 on every row of the warp (the running max did not move): skip the rescale
+      if (__all_sync(0xffffffffu, alpha == 1.f)) {
 #pragma unroll
-      for (int k = 0; k < kBN / 32; ++k)
-        mma_i8(tO, sdesc(pa + 32 * k, 512, 4), sdesc(va + 32 * k, 512, 4), ID_PV, k > 0);
-      mma_commit(bar);
-    }
-    if (!mbar_wait(bar, phase, p.timeout_ns)) *sAbort = 1;
-    phase ^= 1;
-    __syncthreads();
-    if (*sAbort) { aborted = true; break; }
-    tc_fence_after();
-
+        for (int cb = 0; cb < D / 32; ++cb) {
+          uint32_t a[32];
+          tmem_ld32(tPV + 32 * cb, a);
+          tmem_ld_wait();
 #pragma unroll
-    for (int j = 0; j < D / 32; ++j) {
-      uint32_t a[32];
-      tmem_ld32(tO + t_lane + 32 * j, a);
-      tmem_ld_wait();
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 s4 = *reinterpret_cast<const float4*>(sv + 32 * cb + 4 * k4);
+            const int c = 32 * cb + 4 * k4;
+            O[c] = __fmaf_rn(s4.x, __uint_as_float(a[4 * k4]), O[c]);
+            O[c + 1] = __fmaf_rn(s4.y, __uint_as_float(a[4 * k4 + 1]), O[c + 1]);
+            O[c + 2] = __fmaf_rn(s4.z, __uint_as_float(a[4 * k4 + 2]), O[c + 2]);
+            O[c + 3] = __fmaf_rn(s4.w, __uint_as_float(a[4 * k4 + 3]), O[c + 3]);
+          }
+        }
+      } else {
 #pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        const float sv = sVs[32 * j + t];
-        O[32 * j + t] = __fmaf_rn(O[32 * j + t], alpha, sv * static_cast<float>(static_cast<int32_t>(a[t])));
+        for (int cb = 0; cb < D / 32; ++cb) {
+          uint32_t a[32];
+          tmem_ld32(tPV + 32 * cb, a);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 s4 = *reinterpret_cast<const float4*>(sv + 32 * cb + 4 * k4);
+            const int c = 32 * cb + 4 * k4;
+            O[c] = __fmaf_rn(O[c], alpha, s4.x * __uint_as_float(a[4 * k4]));
+            O[c + 1] = __fmaf_rn(O[c + 1], alpha, s4.y * __uint_as_float(a[4 * k4 + 1]));
+            O[c + 2] = __fmaf_rn(O[c + 2], alpha, s4.z * __uint_as_float(a[4 * k4 + 2]));
+            O[c + 3] = __fmaf_rn(O[c + 3], alpha, s4.w * __uint_as_float(a[4 * k4 + 3]));
+          }
+        }
       }
-    }
-    tc_fence_before();
-    __syncthreads();
-  }
+      {
+        uint32_t a[32];
+        tmem_ld32(tPV + D, a);
+        tmem_ld_wait();
+        l = __fmaf_rn(l, alpha, __uint_as_float(a[0]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&pv_empty[t]);
+        mbar_arrive(&op_empty[i % kOps]);
+      }
+      return true;
+    };
 
-  if (!aborted && row < p.N) {
-    const float inv_l = 1.f / l;
-    float4* dst = reinterpret_cast<float4*>(p.out + (head * p.N + row) * D);
+    float sk_next = __ldg(ksc);
+    for (int j = 0; j < nkb; ++j) {
+      const float sk = sk_next;
+      if (j + 1 < nkb) sk_next = __ldg(ksc + j + 1);
+      if (!warp_wait(&s_full[t], j & 1, lim)) { aborted = true; break; }
+      tc_fence_after();
+
+      // ---- running max over the block (first pass over S), then P codes (second pass) ----
+      const int nvalid = min(kBN, p.N - j * kBN);
+      const float c = __fmul_rn(__fmul_rn(sq, sk), p.kappa);
+      const float c18 = c * 262144.f;  // S here is S_int * 2^-18; c * 2^18 is exact
+      float smax = -INFINITY;
 #pragma unroll
-    for (int c4 = 0; c4 < D / 4; ++c4)
-      dst[c4] = make_float4(O[4 * c4] * inv_l, O[4 * c4 + 1] * inv_l, O[4 * c4 + 2] * inv_l, O[4 * c4 + 3] * inv_l);
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t sr[32];
+        tmem_ld32(tS + 32 * hf, sr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (32 * hf + k < nvalid) smax = fmaxf(smax, __uint_as_float(sr[k]));
+      }
+      const float m_new = fmaxf(m, __fmul_rn(smax, c18));
+      const float alpha = ex2_approx(m - m_new);  // 0 on the first block (m = -inf)
+      m = m_new;
+      uint32_t pw[kBN / 4];
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t sr[32];
+        tmem_ld32(tS + 32 * hf, sr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+          float u[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int k = 32 * hf + 4 * k4 + e;
+            u[e] = k < nvalid ? pcode_f(__fmaf_rn(__uint_as_float(sr[4 * k4 + e]), c18, -m), sTau) : 0.f;
+          }
+          pw[8 * hf + k4] = pack_e4m3x4(u[0], u[1], u[2], u[3]);
+          if (DUMP && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr) {
+            const size_t base = (size_t)(row - p.dbg_r0) * p.N + (size_t)j * kBN;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int k = 32 * hf + 4 * k4 + e;
+              if (k < nvalid) {
+                p.s_dump[base + k] = static_cast<int32_t>(__uint_as_float(sr[4 * k4 + e]) * 262144.f);
+                p.p_dump[base + k] = static_cast<uint8_t>(u[e]);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[t]);
+
+      // ---- P codes of this block -> shared memory (buffer j & 1) for the P V MMA;
+      // the other buffer may still feed P V of block j - 1 ----
+      {
+        uint8_t* sP = sP0 + (j & 1) * L::P_BYTES;
+#pragma unroll
+        for (int k = 0; k < kBN / 16; ++k)
+          *reinterpret_cast<uint4*>(sP + swz<64>(r, 16 * k)) =
+              make_uint4(pw[4 * k], pw[4 * k + 1], pw[4 * k + 2], pw[4 * k + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[2 * t + (j & 1)]);
+      }
+
+      // ---- O update of the previous block (its P V is done by now) ----
+      if (j > 0 && !o_update(j - 1, alpha_prev)) { aborted = true; break; }
+      alpha_prev = alpha;
+      if (warp_flag(sAbort)) { aborted = true; break; }
+    }
+    if (!aborted && !o_update(nkb - 1, alpha_prev)) aborted = true;
+    if (aborted) *sAbort = 1;
+
+    if (!aborted && row < p.N) {
+      const float inv_l = 1.f / l;
+      float4* dst = reinterpret_cast<float4*>(p.out + (head * p.N + row) * D);
+#pragma unroll
+      for (int c4 = 0; c4 < D / 4; ++c4)
+        dst[c4] = make_float4(O[4 * c4] * inv_l, O[4 * c4 + 1] * inv_l, O[4 * c4 + 2] * inv_l, O[4 * c4 + 3] * inv_l);
+    }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }

@@ -121,6 +121,17 @@ __device__ __forceinline__ int quant_code(float y, float inv) {
   return max(-7, min(7, c));
 }
 
+// Sign-magnitude nibble of a code in [-7, 7]: bit 3 = sign, bits 0-2 = |v|.
+__device__ __forceinline__ uint32_t nibble(int c) { return static_cast<uint32_t>(c < 0 ? 8 - c : c); }
+
+// Eight codes -> one packed word: byte j holds element j (low nibble) and j+4 (high).
+__device__ __forceinline__ uint32_t pack8(const int (&c)[8]) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) w |= (nibble(c[j]) | (nibble(c[j + 4]) << 4)) << (8 * j);
+  return w;
+}
+
 // fp16 tile [64, D] of one (head, block) -> fp32 smem rows of stride D+1.
 template <int D>
 __device__ __forceinline__ void load_tile(const __half* src, int n0, int N, float* X) {
@@ -240,9 +251,11 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(const Prolog
       uint32_t w[2] = {0u, 0u};
       if (n0 + r < p.N) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t c = static_cast<uint32_t>(quant_code(xr[j], inv)) & 0xFu;
-          w[j >> 3] |= c << (4 * (j & 7));
+        for (int g = 0; g < 2; ++g) {
+          int c[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) c[j] = quant_code(xr[8 * g + j], inv);
+          w[g] = pack8(c);
         }
       }
       *reinterpret_cast<uint2*>(cdst + (size_t)r * (D / 2) + ch * 8) = make_uint2(w[0], w[1]);
@@ -263,14 +276,13 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(const Prolog
     uint32_t w[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      uint32_t acc = 0;
+      int cs[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
         const int r = 8 * j + t;
-        const uint32_t code = (n0 + r < p.N) ? (static_cast<uint32_t>(quant_code(X[r * LD + c], inv)) & 0xFu) : 0u;
-        acc |= code << (4 * t);
+        cs[t] = (n0 + r < p.N) ? quant_code(X[r * LD + c], inv) : 0;
       }
-      w[j] = acc;
+      w[j] = pack8(cs);
     }
     uint4* dst = reinterpret_cast<uint4*>(p.v_codes + ((head * p.nblk + blk) * D + c) * 32);
     dst[0] = make_uint4(w[0], w[1], w[2], w[3]);

@@ -84,6 +84,24 @@ int select_heads(const rota_attn_desc* d, const uint8_t* flags, int want, int16_
   return n;
 }
 
+// The INT4 kernel re-balances registers between its warpgroups with
+// setmaxnreg; that only works if the build gave it exactly the register count
+// the split was designed for, so any other count is refused before launch.
+template <typename K>
+rota_status launch_int4_kernel(K kernel, int smem, dim3 grid, cudaStream_t s, const rota::Int4Params& p) {
+  cudaFuncAttributes fa{};
+  rota_status st = cuda_status(cudaFuncGetAttributes(&fa, kernel));
+  if (st != ROTA_OK) return st;
+  if (fa.numRegs != rota::kLaunchRegs) {
+    std::fprintf(stderr, "rota_attn: INT4 kernel built with %d registers/thread, expected %d; not launching\n",
+                 fa.numRegs, rota::kLaunchRegs);
+    return ROTA_ERR_UNSUPPORTED;
+  }
+  if ((st = set_smem(kernel, smem)) != ROTA_OK) return st;
+  kernel<<<grid, rota::kInt4Threads, smem, s>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
 }  // namespace
 
 extern "C" {
@@ -282,28 +300,15 @@ static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers*
     p.nheads = select_heads(d, head_flags, 0, p.heads);
     if (p.nheads == 0) return ROTA_OK;
   }
-  const dim3 grid((d->N + rota::kBM - 1) / rota::kBM, p.nheads, batches);
+  const dim3 grid((d->N + rota::kRowsPerCta - 1) / rota::kRowsPerCta, p.nheads, batches);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d->head_dim == 128) {
-    using L = rota::Int4Smem<128>;
-    if (dump) {
-      if ((st = set_smem(rota::attn_int4_kernel<128, true>, L::ALLOC)) != ROTA_OK) return st;
-      rota::attn_int4_kernel<128, true><<<grid, rota::kInt4Threads, L::ALLOC, s>>>(p);
-    } else {
-      if ((st = set_smem(rota::attn_int4_kernel<128, false>, L::ALLOC)) != ROTA_OK) return st;
-      rota::attn_int4_kernel<128, false><<<grid, rota::kInt4Threads, L::ALLOC, s>>>(p);
-    }
-  } else {
-    using L = rota::Int4Smem<64>;
-    if (dump) {
-      if ((st = set_smem(rota::attn_int4_kernel<64, true>, L::ALLOC)) != ROTA_OK) return st;
-      rota::attn_int4_kernel<64, true><<<grid, rota::kInt4Threads, L::ALLOC, s>>>(p);
-    } else {
-      if ((st = set_smem(rota::attn_int4_kernel<64, false>, L::ALLOC)) != ROTA_OK) return st;
-      rota::attn_int4_kernel<64, false><<<grid, rota::kInt4Threads, L::ALLOC, s>>>(p);
-    }
-  }
-  return cuda_status(cudaGetLastError());
+  if (d->head_dim == 128)
+    st = dump ? launch_int4_kernel(rota::attn_int4_kernel<128, true>, rota::Int4Smem<128>::ALLOC, grid, s, p)
+              : launch_int4_kernel(rota::attn_int4_kernel<128, false>, rota::Int4Smem<128>::ALLOC, grid, s, p);
+  else
+    st = dump ? launch_int4_kernel(rota::attn_int4_kernel<64, true>, rota::Int4Smem<64>::ALLOC, grid, s, p)
+              : launch_int4_kernel(rota::attn_int4_kernel<64, false>, rota::Int4Smem<64>::ALLOC, grid, s, p);
+  return st;
 }
 
 rota_status rota_attn_fwd_int4(const rota_attn_desc* d, const rota_attn_buffers* buf, const uint8_t* head_flags,

@@ -70,6 +70,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// Warp-collective wait: every lane waits, and the warp leaves with one
+// decision (true only if all lanes saw the phase complete), converged.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Warp-uniform read of a CTA abort flag.
+__device__ __forceinline__ bool warp_flag(volatile int* f) { return __any_sync(0xffffffffu, *f != 0); }
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -132,7 +142,8 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t sbo, uint32_t
 }
 
 // Instruction descriptor: D format (0 f16, 1 f32, 2 s32), A/B formats (kind::i8:
-// 0 u8, 1 s8; kind::f16: 0 f16, 1 bf16), K-major A and B, M x N.
+// 0 u8, 1 s8; kind::f16: 0 f16, 1 bf16; kind::f8f6f4: 0 e4m3), K-major A and
+// B, M x N.
 __host__ __device__ constexpr uint32_t idesc(uint32_t dfmt, uint32_t afmt, uint32_t bfmt, uint32_t M,
                                              uint32_t N, uint32_t b_mn_major = 0) {
   return (dfmt << 4) | (afmt << 7) | (bfmt << 10) | (b_mn_major << 16) | ((N >> 3) << 17) |
@@ -153,6 +164,15 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(id), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(id), "r"(acc)
       : "memory");
 }
@@ -201,19 +221,13 @@ __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t kbyte) {
   return lin ^ (((lin >> 7) & mask) << 4);
 }
 
-// Eight packed s4 codes (low nibble first) -> eight s8 bytes (two words).
-__device__ __forceinline__ void s4x8_to_s8(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  // sign-extend each nibble: (x ^ 8) - 8 per byte
-  const uint32_t even = w & 0x0F0F0F0Fu;          // nibbles 0,2,4,6 -> bytes
-  const uint32_t odd = (w >> 4) & 0x0F0F0F0Fu;    // nibbles 1,3,5,7
-  const uint32_t e = ((even ^ 0x08080808u) | 0x80808080u) - 0x08080808u;
-  const uint32_t o = ((odd ^ 0x08080808u) | 0x80808080u) - 0x08080808u;
-  // bytes of e/o now hold (x^8) - 8 + 0x80 per byte without borrow; remove the 0x80 bias
-  const uint32_t es = e ^ 0x80808080u;
-  const uint32_t os = o ^ 0x80808080u;
-  // interleave: element order n0 n1 n2 n3 | n4 n5 n6 n7 = e0 o0 e1 o1 | e2 o2 e3 o3
-  lo = __byte_perm(es, os, 0x5140);
-  hi = __byte_perm(es, os, 0x7362);
+// One packed word of eight codes (byte j: element j in the low nibble,
+// element j+4 in the high nibble; sign-magnitude nibbles) -> the eight codes
+// as e4m3 subnormals v * 2^-9 (sign bit 7, magnitude in the mantissa bits
+// 0-2, exponent 0), elements 0-3 in `lo` and 4-7 in `hi`.  Exact for |v| <= 7.
+__device__ __forceinline__ void codes8_to_e4m3(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  lo = (w & 0x07070707u) | ((w & 0x08080808u) << 4);
+  hi = ((w >> 4) & 0x07070707u) | (w & 0x80808080u);
 }
 
 }  // namespace rota
