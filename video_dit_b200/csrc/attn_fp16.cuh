@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(kF16Threads, 1) attn_fp16_kernel(const __grid_
       uint32_t r0[32], r1[32];
       tmem_ld32(tS + t_lane, r0);
       tmem_ld32(tS + t_lane + 32, r1);
-      tmem_ld_wait();
+      tmem_wait_dep2(r0, r1);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         s[j] = __uint_as_float(r0[j]) * p.scale_log2;
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(kF16Threads, 1) attn_fp16_kernel(const __grid_
     for (int j = 0; j < D / 32; ++j) {
       uint32_t a[32];
       tmem_ld32(tO + t_lane + 32 * j, a);
-      tmem_ld_wait();
+      tmem_wait_dep(a);
 #pragma unroll
       for (int t = 0; t < 32; ++t) O[32 * j + t] = __fmaf_rn(O[32 * j + t], alpha, __uint_as_float(a[t]));
     }

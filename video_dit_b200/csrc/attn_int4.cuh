@@ -386,46 +386,41 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       if (!warp_wait(&op_full[i % kOps], (i / kOps) & 1, lim)) return false;
       tc_fence_after();
       const float* sv = sSv + (i % kOps) * D;
-      // alpha == 1 on every row of the warp (the running max did not move): skip the rescale
-      if (__all_sync(0xffffffffu, alpha == 1.f)) {
+      // alpha == 1 on every row of the warp (the running max did not move): no rescale
+      const bool unit = __all_sync(0xffffffffu, alpha == 1.f);
 #pragma unroll
-        for (int cb = 0; cb < D / 32; ++cb) {
-          uint32_t a[32];
-          tmem_ld32(tPV + 32 * cb, a);
-          tmem_ld_wait();
+      for (int cb = 0; cb < D / 64; ++cb) {
+        uint32_t a[64];
+        uint32_t(&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&a[0]);
+        uint32_t(&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&a[32]);
+        tmem_ld32(tPV + 64 * cb, a0);
+        tmem_ld32(tPV + 64 * cb + 32, a1);
+        tmem_wait_dep2(a0, a1);
+        if (unit) {
 #pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 s4 = *reinterpret_cast<const float4*>(sv + 32 * cb + 4 * k4);
-            const int c = 32 * cb + 4 * k4;
-            O[c] = __fmaf_rn(s4.x, __uint_as_float(a[4 * k4]), O[c]);
-            O[c + 1] = __fmaf_rn(s4.y, __uint_as_float(a[4 * k4 + 1]), O[c + 1]);
-            O[c + 2] = __fmaf_rn(s4.z, __uint_as_float(a[4 * k4 + 2]), O[c + 2]);
-            O[c + 3] = __fmaf_rn(s4.w, __uint_as_float(a[4 * k4 + 3]), O[c + 3]);
+          for (int k4 = 0; k4 < 16; ++k4) {
+            const float4 s4 = *reinterpret_cast<const float4*>(sv + 64 * cb + 4 * k4);
+            const int c = 64 * cb + 4 * k4;
+            fma2(O[c], O[c + 1], s4.x, s4.y, __uint_as_float(a[4 * k4]), __uint_as_float(a[4 * k4 + 1]), O[c], O[c + 1]);
+            fma2(O[c + 2], O[c + 3], s4.z, s4.w, __uint_as_float(a[4 * k4 + 2]), __uint_as_float(a[4 * k4 + 3]),
+                 O[c + 2], O[c + 3]);
           }
-        }
-      } else {
+        } else {
 #pragma unroll
-        for (int cb = 0; cb < D / 32; ++cb) {
-          uint32_t a[32];
-          tmem_ld32(tPV + 32 * cb, a);
-          tmem_ld_wait();
-#pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 s4 = *reinterpret_cast<const float4*>(sv + 32 * cb + 4 * k4);
-            const int c = 32 * cb + 4 * k4;
-            O[c] = __fmaf_rn(O[c], alpha, s4.x * __uint_as_float(a[4 * k4]));
-            O[c + 1] = __fmaf_rn(O[c + 1], alpha, s4.y * __uint_as_float(a[4 * k4 + 1]));
-            O[c + 2] = __fmaf_rn(O[c + 2], alpha, s4.z * __uint_as_float(a[4 * k4 + 2]));
-            O[c + 3] = __fmaf_rn(O[c + 3], alpha, s4.w * __uint_as_float(a[4 * k4 + 3]));
+          for (int k4 = 0; k4 < 16; ++k4) {
+            const float4 s4 = *reinterpret_cast<const float4*>(sv + 64 * cb + 4 * k4);
+            const int c = 64 * cb + 4 * k4;
+            float x0, x1, x2, x3;
+            mul2(x0, x1, s4.x, s4.y, __uint_as_float(a[4 * k4]), __uint_as_float(a[4 * k4 + 1]));
+            mul2(x2, x3, s4.z, s4.w, __uint_as_float(a[4 * k4 + 2]), __uint_as_float(a[4 * k4 + 3]));
+            fma2(O[c], O[c + 1], O[c], O[c + 1], alpha, alpha, x0, x1);
+            fma2(O[c + 2], O[c + 3], O[c + 2], O[c + 3], alpha, alpha, x2, x3);
           }
         }
       }
-      {
-        uint32_t a[32];
-        tmem_ld32(tPV + D, a);
-        tmem_ld_wait();
-        l = __fmaf_rn(l, alpha, __uint_as_float(a[0]));
-      }
+      uint32_t lsum = tmem_ld1(tPV + D);
+      tmem_wait_dep1(lsum);
+      l = __fmaf_rn(l, alpha, __uint_as_float(lsum));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -435,54 +430,79 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       return true;
     };
 
+    constexpr float kMagic = 12582912.f;          // 1.5 * 2^23: x + kMagic rounds x to an integer
+    constexpr float kNear = 0.5f - 1e-4f;         // |15 e - rne(15 e)| above this: decide exactly
     float sk_next = __ldg(ksc);
     for (int j = 0; j < nkb; ++j) {
       const float sk = sk_next;
       if (j + 1 < nkb) sk_next = __ldg(ksc + j + 1);
       if (!warp_wait(&s_full[t], j & 1, lim)) { aborted = true; break; }
       tc_fence_after();
+      uint32_t sr[kBN];
+      {
+        uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+        uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+        tmem_ld32(tS, s0);
+        tmem_ld32(tS + 32, s1);
+        tmem_wait_dep2(s0, s1);
+      }
 
-      // ---- running max over the block (first pass over S), then P codes (second pass) ----
+      // ---- running max over the block's valid keys ----
       const int nvalid = min(kBN, p.N - j * kBN);
       const float c = __fmul_rn(__fmul_rn(sq, sk), p.kappa);
       const float c18 = c * 262144.f;  // S here is S_int * 2^-18; c * 2^18 is exact
       float smax = -INFINITY;
+      if (nvalid == kBN) {
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t sr[32];
-        tmem_ld32(tS + 32 * hf, sr);
-        tmem_ld_wait();
+        for (int k = 0; k < kBN; k += 2) smax = max3(smax, __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
+      } else {
 #pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (32 * hf + k < nvalid) smax = fmaxf(smax, __uint_as_float(sr[k]));
+        for (int k = 0; k < kBN; ++k)
+          if (k < nvalid) smax = fmaxf(smax, __uint_as_float(sr[k]));
       }
       const float m_new = fmaxf(m, __fmul_rn(smax, c18));
       const float alpha = ex2_approx(m - m_new);  // 0 on the first block (m = -inf)
       m = m_new;
+
+      // ---- P codes u = rne(15 * 2^(S c - m)): branch-free estimate for all 64 keys ----
       uint32_t pw[kBN / 4];
+      float near = 0.f;
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t sr[32];
-        tmem_ld32(tS + 32 * hf, sr);
-        tmem_ld_wait();
+      for (int k = 0; k < kBN; k += 4) {
+        float d0, d1, d2, d3, r0, r1, r2, r3, f0, f1, f2, f3;
+        fma2(d0, d1, __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]), c18, c18, -m, -m);
+        fma2(d2, d3, __uint_as_float(sr[k + 2]), __uint_as_float(sr[k + 3]), c18, c18, -m, -m);
+        const float e0 = ex2_approx(d0), e1 = ex2_approx(d1), e2 = ex2_approx(d2), e3 = ex2_approx(d3);
+        fma2(f0, f1, e0, e1, 15.f, 15.f, kMagic, kMagic);     // kMagic + rne(15 e)
+        fma2(f2, f3, e2, e3, 15.f, 15.f, kMagic, kMagic);
+        add2(r0, r1, f0, f1, -kMagic, -kMagic);                // rne(15 e), exact
+        add2(r2, r3, f2, f3, -kMagic, -kMagic);
+        fma2(f0, f1, e0, e1, 15.f, 15.f, -r0, -r1);            // 15 e - rne(15 e)
+        fma2(f2, f3, e2, e3, 15.f, 15.f, -r2, -r3);
+        near = max3(near, fabsf(f0), fabsf(f1));
+        near = max3(near, fabsf(f2), fabsf(f3));
+        pw[k / 4] = pack_e4m3x4(r0, r1, r2, r3);
+      }
+      uint8_t* sP = sP0 + (j & 1) * L::P_BYTES;
 #pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-          float u[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int k = 32 * hf + 4 * k4 + e;
-            u[e] = k < nvalid ? pcode_f(__fmaf_rn(__uint_as_float(sr[4 * k4 + e]), c18, -m), sTau) : 0.f;
-          }
-          pw[8 * hf + k4] = pack_e4m3x4(u[0], u[1], u[2], u[3]);
-          if (DUMP && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr) {
-            const size_t base = (size_t)(row - p.dbg_r0) * p.N + (size_t)j * kBN;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int k = 32 * hf + 4 * k4 + e;
-              if (k < nvalid) {
-                p.s_dump[base + k] = static_cast<int32_t>(__uint_as_float(sr[4 * k4 + e]) * 262144.f);
-                p.p_dump[base + k] = static_cast<uint8_t>(u[e]);
-              }
+      for (int k = 0; k < kBN / 16; ++k)
+        *reinterpret_cast<uint4*>(sP + swz<64>(r, 16 * k)) =
+            make_uint4(pw[4 * k], pw[4 * k + 1], pw[4 * k + 2], pw[4 * k + 3]);
+
+      // ---- exact decisions (rare): estimates within 1e-4 of a half-integer, masked keys ----
+      const bool fix = near > kNear;
+      if (__any_sync(0xffffffffu, fix) || nvalid < kBN || DUMP) {
+#pragma unroll 1
+        for (int k = 0; k < kBN; ++k) {
+          uint32_t sbits = tmem_ld1(tS + k);
+          tmem_wait_dep1(sbits);
+          const float sk_ = __uint_as_float(sbits);
+          if (fix || k >= nvalid || DUMP) {
+            const float u = k < nvalid ? pcode_f(__fmaf_rn(sk_, c18, -m), sTau) : 0.f;
+            sP[swz<64>(r, k)] = static_cast<uint8_t>(pack_e4m3x4(u, 0.f, 0.f, 0.f) & 0xFFu);
+            if (DUMP && k < nvalid && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr) {
+              const size_t base = (size_t)(row - p.dbg_r0) * p.N + (size_t)j * kBN;
+              p.s_dump[base + k] = static_cast<int32_t>(sk_ * 262144.f);
             }
           }
         }
@@ -490,18 +510,17 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[t]);
-
-      // ---- P codes of this block -> shared memory (buffer j & 1) for the P V MMA;
-      // the other buffer may still feed P V of block j - 1 ----
-      {
-        uint8_t* sP = sP0 + (j & 1) * L::P_BYTES;
-#pragma unroll
-        for (int k = 0; k < kBN / 16; ++k)
-          *reinterpret_cast<uint4*>(sP + swz<64>(r, 16 * k)) =
-              make_uint4(pw[4 * k], pw[4 * k + 1], pw[4 * k + 2], pw[4 * k + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[2 * t + (j & 1)]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[2 * t + (j & 1)]);
+      if (DUMP && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr) {
+        // P codes as the MMA will read them, decoded from the e4m3 bytes
+        const size_t base = (size_t)(row - p.dbg_r0) * p.N + (size_t)j * kBN;
+        for (int k = 0; k < nvalid; ++k) {
+          const uint32_t b = sP[swz<64>(r, k)];
+          const uint32_t e = (b >> 3) & 15u, mt = b & 7u;
+          p.p_dump[base + k] = static_cast<uint8_t>(b == 0 ? 0 : ((8u + mt) << e) >> 10);
+        }
       }
 
       // ---- O update of the previous block (its P V is done by now) ----
