@@ -78,6 +78,11 @@ typedef struct {
  *                      (may be NULL when no head is flagged)
  *   rope_cos, rope_sin: fp32 tables from rota_attn_build_rope_tables, copied
  *                      to the device by the caller.
+ *   int4_work        : workspace of rota_attn_fwd_int4 (bytes[ROTA_BUF_INT4_WORK]):
+ *                      the K and V codes of the INT4 heads widened once per call
+ *                      into the 8-bit tensor-core operand tiles (pre-swizzled
+ *                      e4m3 images) and the V scales times 2^9.  Transient: its
+ *                      contents are rewritten by every call.
  */
 typedef struct {
   uint8_t* q_codes;
@@ -90,6 +95,7 @@ typedef struct {
   uint16_t* k_rope;
   const float* rope_cos;
   const float* rope_sin;
+  uint8_t* int4_work;
 } rota_attn_buffers;
 
 /* Indices into the `bytes` array of rota_attn_buffer_sizes. */
@@ -103,6 +109,7 @@ enum {
   ROTA_BUF_Q_ROPE,
   ROTA_BUF_K_ROPE,
   ROTA_BUF_ROPE_TABLE, /* each of rope_cos and rope_sin */
+  ROTA_BUF_INT4_WORK,
   ROTA_BUF_COUNT
 };
 
@@ -149,7 +156,9 @@ rota_status rota_attn_prepare_qk(const rota_attn_desc* desc, const uint16_t* q, 
  * in 0..15 (fixed scale 1/15, zero-point 0: the whole unsigned 4-bit range,
  * as the abstract's "Range-optimized P Quantization" asks); integer P V on
  * the tensor cores per 64-key block; V scales, rescaling by 2^(m_old - m_new)
- * and the row sum of the codes in fp32; out = O / l.
+ * and the row sum of the codes in fp32; out = O / l.  Two launches: the K / V
+ * codes are first widened once into buf->int4_work, then the attention kernel
+ * streams the widened tiles with TMA bulk copies.
  *   out: fp32 [B,H,N,head_dim]; rows of flagged heads are not written.
  */
 rota_status rota_attn_fwd_int4(const rota_attn_desc* desc, const rota_attn_buffers* buf,
@@ -184,8 +193,8 @@ const char* rota_attn_status_string(rota_status s);
  * every head takes the INT4 path (no FP16 fallback).  The intermediate codes,
  * scales and RoPE tables live in one 16 MiB array in the library's static
  * device memory, which every GPU that loads the library holds until exit.
- * Its size bounds the problem: B*H*nblk*(96*head_dim + 4*head_dim + 8) bytes
- * of codes and scales plus the RoPE tables (each entry padded to 256 bytes)
+ * Its size bounds the problem: B*H*nblk*(232*head_dim + 8) bytes of codes,
+ * widened tiles and scales plus the RoPE tables (each entry padded to 256 bytes)
  * must fit in ROTA_NOALLOC_SCRATCH_BYTES, and each RoPE table in
  * ROTA_NOALLOC_MAX_TABLE floats; larger problems return
  * ROTA_ERR_UNSUPPORTED, with nothing enqueued.

@@ -102,7 +102,9 @@ def test_pcode_function_matches_oracle_dense():
 
 
 def test_pcode_function_exhaustive_near_thresholds():
-    """Every fp32 within 2^16 ulps of each of the 15 code thresholds."""
+    """Every fp32 within 2^16 ulps of each of the 15 code thresholds: the
+    band in which the kernel re-decides a code exactly must cover every
+    estimate that could round the wrong way."""
     import torch
     from gpu_util import lib
     ra = lib()
@@ -133,3 +135,38 @@ def test_int4_long_sequence_sampled_rows():
     assert e <= TOL, (e, rel, cos)
     o0 = oracle.attn_int4(ref, w.N, sm_scale(w), 0, 0, 0, 64)          # first rows of the other head
     assert row_stats(out[0, 0, :64], o0)[0] <= TOL
+
+
+def test_pcode_function_exhaustive_range():
+    """Every fp32 d in [-6, -0] (about 1.1e9 values): the kernel's P-code
+    function against the oracle's, via the oracle's own decision boundaries
+    (u(d) is a step function of d, so 15 boundary values pin it everywhere)."""
+    import torch
+    from gpu_util import lib
+    ra = lib()
+    lo, hi = 0x80000000, 0xC0C00000            # bit patterns of -0.0 and -6.0; value falls as bits rise
+
+    def val(bits):
+        return float(np.uint32(bits).view(np.float32))
+    taus = []
+    for kk in range(1, 16):                     # most negative d whose oracle code is still >= kk
+        a, b = lo, hi                            # code(a) >= kk > code(b)
+        while b - a > 1:
+            mid = (a + b) // 2
+            if oracle.pcode(val(mid)) >= kk:
+                a = mid
+            else:
+                b = mid
+        taus.append(val(a))
+    tau = torch.tensor(sorted(taus), dtype=torch.float32, device="cuda")
+    chunk = 1 << 27
+    u = torch.empty(chunk, dtype=torch.uint8, device="cuda")
+    for b0 in range(lo, hi + 1, chunk):
+        n = min(chunk, hi + 1 - b0)
+        bits = torch.arange(b0 - (1 << 32), b0 - (1 << 32) + n, dtype=torch.int32, device="cuda")
+        d = bits.view(torch.float32)
+        ra._check(ra.rota_attn_debug_pcode(d, u[:n]), "pcode")
+        want = torch.bucketize(d, tau, right=True).to(torch.uint8)
+        bad = (u[:n] != want).nonzero()
+        assert bad.numel() == 0, (b0, d[bad[:5, 0]].cpu().numpy(), u[bad[:5, 0]].cpu().numpy(),
+                                  want[bad[:5, 0]].cpu().numpy())

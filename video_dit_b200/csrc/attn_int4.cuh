@@ -14,12 +14,16 @@
 // 2^-9 hold exactly -- the same integers an s32 accumulation gives, already
 // in fp32 for the softmax and the V scales.
 //
+// The packed K / V nibbles are widened once per call by widen_kv_kernel into
+// the exact shared-memory images of the operand tiles (swizzled K-major e4m3),
+// so the main loop moves them with plain TMA bulk copies; widening inside the
+// main loop would repeat the same work in every CTA of a head.
+//
 // One CTA = two 128-row query tiles of one head (256 rows), 384 threads:
-//   warp 0      TMA producer: packed K / V codes and V scales of each 64-key
-//               block -> a 4-slot shared-memory staging ring (cp.async.bulk);
+//   warp 0      TMA producer: widened K / V^T tiles and V scales of each 64-key
+//               block -> a 4-stage shared-memory ring (cp.async.bulk);
 //   warp 1      TMEM owner and MMA issuer (one thread);
-//   warps 2-3   widen the staged nibbles into the swizzled K-major e4m3 K and
-//               V^T operand tiles (3 stages) -- once per block for both tiles;
+//   warps 2-3   fill the constant rows once, then idle;
 //   warps 4-7   query tile 0, warps 8-11 query tile 1 (thread = row = TMEM lane):
 //               running max, P codes, O update, epilogue.
 // Per 64-key block j and tile t the MMA warp issues S_t = Q_t K_j^T (128 x 64)
@@ -43,6 +47,7 @@ struct Int4Params {
   const float* k_scale;
   const uint8_t* v_codes;
   const float* v_scale;
+  const uint8_t* work;  // widened K / V^T tiles + 512 * v_scale per (head, block)
   float* out;
   int H, N, nblk;
   float kappa;          // RN(sm_scale * log2 e)
@@ -59,8 +64,7 @@ struct Int4Params {
 
 constexpr int kInt4Threads = 384;
 constexpr int kRowsPerCta = 2 * kBM;
-constexpr int kStg = 4;   // staging slots
-constexpr int kOps = 3;   // widened operand stages
+constexpr int kOps = 4;   // operand stages
 constexpr int kProducerRegs = 40;
 constexpr int kConsumerRegs = 232;
 // Register split: kProducerRegs * 128 + kConsumerRegs * 256 equals the launch
@@ -75,24 +79,22 @@ struct Int4Smem {
   static constexpr int ROWB = D;              // bytes per e4m3 Q / K row
   static constexpr uint32_t LAYOUT_QK = D == 128 ? 2u : 4u;  // 128B / 64B swizzle
   static constexpr uint32_t SBO_QK = 8 * D;
-  static constexpr int KPACK = kBN * D / 2;
-  static constexpr int VPACK = D * kBN / 2;
-  static constexpr int STG_BYTES = KPACK + VPACK + D * 4;
   static constexpr int Q_BYTES = kBM * D;
   static constexpr int K_BYTES = kBN * D;
+  static constexpr int VIMG_BYTES = D * kBN;                      // widened V^T rows 0..D-1
   static constexpr int V_BYTES = ((NPV * kBN + 1023) / 1024) * 1024;
   static constexpr int OP_BYTES = K_BYTES + V_BYTES;
+  static constexpr int IMG_BYTES = K_BYTES + VIMG_BYTES + D * 4;  // one block in int4_work
   static constexpr int P_BYTES = kBM * kBN;
   static constexpr int OFF_Q = 0;                              // 2 tiles
   static constexpr int OFF_OP = OFF_Q + 2 * Q_BYTES;           // kOps stages
   static constexpr int OFF_P = OFF_OP + kOps * OP_BYTES;       // 2 tiles x 2 buffers
-  static constexpr int OFF_STG = OFF_P + 4 * P_BYTES;          // kStg slots
-  static constexpr int OFF_SV = OFF_STG + kStg * STG_BYTES;    // kOps x D floats: 512 * v_scale
+  static constexpr int OFF_SV = OFF_P + 4 * P_BYTES;           // kOps x D floats: 512 * v_scale
   static constexpr int OFF_TAU = OFF_SV + kOps * D * 4;
   static constexpr int OFF_BAR = OFF_TAU + 64;
-  // barriers: stg_full[4] stg_empty[4] op_full[3] op_empty[3] s_full[2] s_empty[2]
-  //           pv_full[2] pv_empty[2] q_full mma_done p_full[2 tiles][2 buffers]
-  static constexpr int NBAR = 4 + 4 + 3 + 3 + 2 + 2 + 2 + 2 + 1 + 1 + 4;
+  // barriers: op_full[4] op_empty[4] s_full[2] s_empty[2] pv_full[2] pv_empty[2]
+  //           q_full mma_done p_full[2 tiles][2 buffers]
+  static constexpr int NBAR = 4 + 4 + 2 + 2 + 2 + 2 + 1 + 1 + 4;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int BYTES = OFF_ABORT + 4;
@@ -100,20 +102,26 @@ struct Int4Smem {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S0 = 0, T_S1 = kBN, T_PV0 = 2 * kBN, T_PV1 = 2 * kBN + NPV;
   static_assert(T_PV1 + NPV <= TMEM_COLS, "TMEM budget");
-  static_assert(STG_BYTES % 16 == 0 && KPACK % 16 == 0 && VPACK % 16 == 0, "bulk copy sizes");
+  static_assert(IMG_BYTES % 16 == 0 && K_BYTES % 16 == 0 && VIMG_BYTES % 16 == 0, "bulk copy sizes");
   static_assert(OFF_OP % 1024 == 0 && OP_BYTES % 1024 == 0 && K_BYTES % 1024 == 0 && OFF_P % 1024 == 0,
                 "swizzle atom alignment");
-  static_assert(OFF_STG % 16 == 0 && STG_BYTES % 16 == 0 && OFF_BAR % 8 == 0, "alignment");
+  static_assert(OFF_SV % 16 == 0 && OFF_BAR % 8 == 0, "alignment");
 };
 
 // Range-optimised P code u = rne(15 * 2^d) in exact arithmetic (d <= ~0).
-// The MUFU estimate is within ~4e-6 of 15 * 2^d; only when it falls within
-// 1e-4 of a half-integer is the decision taken by the exact threshold table.
+// The estimate rne(15 e), e = ex2.approx(d), is within ~4e-6 of the exact
+// 15 * 2^d before rounding (ex2.approx: ~2 ulp); only when 15 e lies within
+// 1e-5 of a half-integer is the decision taken by the exact threshold table
+// tau.  (The band is validated exhaustively near every threshold by the tests.)  The main loop runs
+// the same arithmetic (fast estimate for every key, this function for the keys
+// it flags), so this is also the function the exhaustive test checks.
+constexpr float kMagic = 12582912.f;   // 1.5 * 2^23: x + kMagic rounds x to an integer
+constexpr float kNear = 0.5f - 1e-5f;  // |15 e - rne(15 e)| above this: decide exactly
 __device__ __forceinline__ float pcode_f(float d, const float* tau) {
-  const float e = 15.f * ex2_approx(d);
-  float r = __fsub_rn(__fadd_rn(e, 12582912.f), 12582912.f);  // rne to integer
-  const float fr = e - r;
-  if (fabsf(fr) > 0.5f - 1e-4f) {
+  const float e = ex2_approx(d);
+  float r = __fadd_rn(__fmaf_rn(e, 15.f, kMagic), -kMagic);  // rne(15 e)
+  const float fr = __fmaf_rn(e, 15.f, -r);
+  if (fabsf(fr) > kNear) {
     int j = fr > 0.f ? static_cast<int>(r) + 1 : static_cast<int>(r);
     j = max(1, min(15, j));
     r = static_cast<float>(d >= tau[j] ? j : j - 1);
@@ -151,20 +159,18 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-  uint64_t* stg_full = bars;
-  uint64_t* stg_empty = bars + 4;
-  uint64_t* op_full = bars + 8;
-  uint64_t* op_empty = bars + 11;
-  uint64_t* s_full = bars + 14;
-  uint64_t* s_empty = bars + 16;
-  uint64_t* pv_full = bars + 18;
-  uint64_t* pv_empty = bars + 20;
-  uint64_t* q_full = bars + 22;
-  uint64_t* mma_done = bars + 23;
+  uint64_t* op_full = bars;
+  uint64_t* op_empty = bars + 4;
+  uint64_t* s_full = bars + 8;
+  uint64_t* s_empty = bars + 10;
+  uint64_t* pv_full = bars + 12;
+  uint64_t* pv_empty = bars + 14;
+  uint64_t* q_full = bars + 16;
+  uint64_t* mma_done = bars + 17;
   // One barrier per P buffer (tile t, block parity): tile t may write P(j+1)
   // before the MMA warp has waited for P(j), so a single barrier per tile
   // could complete two phases ahead of its waiter.
-  uint64_t* p_full = bars + 24;  // p_full[2 * t + (j & 1)], phase (j >> 1) & 1
+  uint64_t* p_full = bars + 18;  // p_full[2 * t + (j & 1)], phase (j >> 1) & 1
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + L::OFF_ABORT);
   float* sTau = reinterpret_cast<float*>(smem + L::OFF_TAU);
@@ -180,12 +186,8 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
 
   if (tid < 16) sTau[tid] = p.tau[tid];
   if (tid == 0) {
-    for (int i = 0; i < kStg; ++i) {
-      mbar_init(&stg_full[i], 1);
-      mbar_init(&stg_empty[i], 2);
-    }
     for (int i = 0; i < kOps; ++i) {
-      mbar_init(&op_full[i], 2);
+      mbar_init(&op_full[i], 1);
       mbar_init(&op_empty[i], 1 + 8);
     }
     for (int t = 0; t < 2; ++t) {
@@ -196,7 +198,7 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       mbar_init(&pv_full[t], 1);
       mbar_init(&pv_empty[t], 4);
     }
-    mbar_init(q_full, 8);
+    mbar_init(q_full, 8 + 2);
     mbar_init(mma_done, 1);
     *sAbort = 0;
     fence_mbar_init();
@@ -216,22 +218,23 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     setmaxnreg_producer();
     if (warp == 0) {
       if (lane == 0) {
-        // ---- TMA producer ----
+        // ---- TMA producer: widened tiles of block j -> operand stage j % kOps ----
         int issued = 0;
         for (int j = 0; j < nkb; ++j) {
-          const int slot = j % kStg;
-          if (!mbar_wait(&stg_empty[slot], ((j / kStg) & 1) ^ 1, lim)) { *sAbort = 1; break; }
+          const int op = j % kOps;
+          if (!mbar_wait(&op_empty[op], ((j / kOps) & 1) ^ 1, lim)) { *sAbort = 1; break; }
           if (*sAbort) break;
-          uint8_t* dst = smem + L::OFF_STG + slot * L::STG_BYTES;
-          mbar_arrive_expect_tx(&stg_full[slot], L::STG_BYTES);
-          bulk_g2s(dst, p.k_codes + (head * npad + (size_t)j * kBN) * (D / 2), L::KPACK, &stg_full[slot]);
-          bulk_g2s(dst + L::KPACK, p.v_codes + (head * p.nblk + j) * (size_t)D * 32, L::VPACK, &stg_full[slot]);
-          bulk_g2s(dst + L::KPACK + L::VPACK, p.v_scale + (head * p.nblk + j) * D, D * 4, &stg_full[slot]);
+          uint8_t* kt = smem + L::OFF_OP + op * L::OP_BYTES;
+          const uint8_t* src = p.work + (head * p.nblk + j) * (size_t)L::IMG_BYTES;
+          mbar_arrive_expect_tx(&op_full[op], L::K_BYTES + L::VIMG_BYTES + D * 4);
+          bulk_g2s(kt, src, L::K_BYTES, &op_full[op]);
+          bulk_g2s(kt + L::K_BYTES, src + L::K_BYTES, L::VIMG_BYTES, &op_full[op]);
+          bulk_g2s(sSv + op * D, src + L::K_BYTES + L::VIMG_BYTES, D * 4, &op_full[op]);
           issued = j + 1;
         }
         // drain: every issued copy has landed before the CTA may exit
-        for (int j = (issued > kStg ? issued - kStg : 0); j < issued; ++j)
-          mbar_wait(&stg_full[j % kStg], (j / kStg) & 1, lim);
+        for (int j = (issued > kOps ? issued - kOps : 0); j < issued; ++j)
+          mbar_wait(&op_full[j % kOps], (j / kOps) & 1, lim);
       }
     } else if (warp == 1) {
       if (lane == 0) {
@@ -286,57 +289,17 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         mbar_wait(mma_done, 0, lim);
       }
     } else {
-      // ---- widening warps (2, 3): staged nibbles -> e4m3 operand tiles ----
+      // ---- warps 2, 3: the constant ones rows D..D+15 of every V^T stage (e4m3 1.0 = 0x38) ----
       const int wt = tid - 64;  // 0..63
-      // the constant ones rows D..D+15 of every V^T stage (e4m3 1.0 = 0x38)
       for (int op = 0; op < kOps; ++op) {
         uint8_t* vt = smem + L::OFF_OP + op * L::OP_BYTES + L::K_BYTES;
         for (int i = wt; i < 16 * kBN / 16; i += 64)
           *reinterpret_cast<uint4*>(vt + D * kBN + 16 * i) =
               make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
       }
-      for (int j = 0; j < nkb; ++j) {
-        const int slot = j % kStg, op = j % kOps;
-        if (!warp_wait(&stg_full[slot], (j / kStg) & 1, lim)) { *sAbort = 1; break; }
-        if (!warp_wait(&op_empty[op], ((j / kOps) & 1) ^ 1, lim)) { *sAbort = 1; break; }
-        if (warp_flag(sAbort)) break;
-        const uint8_t* sg = smem + L::OFF_STG + slot * L::STG_BYTES;
-        uint8_t* kt = smem + L::OFF_OP + op * L::OP_BYTES;
-        uint8_t* vt = kt + L::K_BYTES;
-        // K: 64 rows x D/2 bytes packed; a 16-byte chunk = 32 channels of one row
-        for (int i = wt; i < kBN * D / 32; i += 64) {
-          const int rr = i / (D / 32), cg = i % (D / 32);
-          const uint4 w = *reinterpret_cast<const uint4*>(sg + 16 * i);
-          uint32_t o[8];
-          codes8_to_e4m3(w.x, o[0], o[1]);
-          codes8_to_e4m3(w.y, o[2], o[3]);
-          codes8_to_e4m3(w.z, o[4], o[5]);
-          codes8_to_e4m3(w.w, o[6], o[7]);
-          *reinterpret_cast<uint4*>(kt + swz<L::ROWB>(rr, cg * 32)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(kt + swz<L::ROWB>(rr, cg * 32 + 16)) = make_uint4(o[4], o[5], o[6], o[7]);
-        }
-        // V: D channel rows x 32 bytes packed (64 keys); a chunk = 32 keys of one channel
-        for (int i = wt; i < D * 2; i += 64) {
-          const int c = i >> 1, hl = i & 1;
-          const uint4 w = *reinterpret_cast<const uint4*>(sg + L::KPACK + 16 * i);
-          uint32_t o[8];
-          codes8_to_e4m3(w.x, o[0], o[1]);
-          codes8_to_e4m3(w.y, o[2], o[3]);
-          codes8_to_e4m3(w.z, o[4], o[5]);
-          codes8_to_e4m3(w.w, o[6], o[7]);
-          *reinterpret_cast<uint4*>(vt + swz<64>(c, hl * 32)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(vt + swz<64>(c, hl * 32 + 16)) = make_uint4(o[4], o[5], o[6], o[7]);
-        }
-        // V scales x 2^9 (the weight of an e4m3-subnormal V code), exact
-        const float* vs = reinterpret_cast<const float*>(sg + L::KPACK + L::VPACK);
-        for (int c = wt; c < D; c += 64) sSv[op * D + c] = vs[c] * 512.f;
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&op_full[op]);
-          mbar_arrive(&stg_empty[slot]);
-        }
-      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_full);
     }
   } else {
     // ===================================================== query-tile warpgroups
@@ -382,7 +345,7 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     // columns carry the sum of the block's P codes for l.
     auto o_update = [&](int i, float alpha) -> bool {
       if (!warp_wait(&pv_full[t], i & 1, lim)) return false;
-      // the V scales of block i were written by the widening warps before op_full
+      // the V scales of block i land with the operand stage (op_full)
       if (!warp_wait(&op_full[i % kOps], (i / kOps) & 1, lim)) return false;
       tc_fence_after();
       const float* sv = sSv + (i % kOps) * D;
@@ -430,8 +393,6 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       return true;
     };
 
-    constexpr float kMagic = 12582912.f;          // 1.5 * 2^23: x + kMagic rounds x to an integer
-    constexpr float kNear = 0.5f - 1e-4f;         // |15 e - rne(15 e)| above this: decide exactly
     float sk_next = __ldg(ksc);
     for (int j = 0; j < nkb; ++j) {
       const float sk = sk_next;
@@ -489,22 +450,52 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         *reinterpret_cast<uint4*>(sP + swz<64>(r, 16 * k)) =
             make_uint4(pw[4 * k], pw[4 * k + 1], pw[4 * k + 2], pw[4 * k + 3]);
 
-      // ---- exact decisions (rare): estimates within 1e-4 of a half-integer, masked keys ----
-      const bool fix = near > kNear;
-      if (__any_sync(0xffffffffu, fix) || nvalid < kBN || DUMP) {
-#pragma unroll 1
+      // ---- exact decisions (rare): estimates within 1e-5 of a half-integer ----
+      // Recompute which keys were near a tie (same arithmetic as above), then
+      // visit only the columns some lane flagged; S is still in TMEM.
+      if (__any_sync(0xffffffffu, near > kNear)) {
+        // S is still in TMEM (s_empty is released below): reload it here so the
+        // fast path above does not have to keep 64 registers alive.
+        uint32_t s2[kBN];
+        {
+          uint32_t(&t0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s2[0]);
+          uint32_t(&t1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s2[32]);
+          tmem_ld32(tS, t0);
+          tmem_ld32(tS + 32, t1);
+          tmem_wait_dep2(t0, t1);
+        }
+        uint32_t mlo = 0, mhi = 0;
+#pragma unroll
+        for (int k = 0; k < kBN; ++k) {
+          const float d = __fmaf_rn(__uint_as_float(s2[k]), c18, -m);
+          const float e = ex2_approx(d);
+          const float rr = __fadd_rn(__fmaf_rn(e, 15.f, kMagic), -kMagic);
+          const bool hit = fabsf(__fmaf_rn(e, 15.f, -rr)) > kNear;
+          if (k < 32) mlo |= static_cast<uint32_t>(hit) << k;
+          else mhi |= static_cast<uint32_t>(hit) << (k - 32);
+        }
+        uint32_t wlo = __reduce_or_sync(0xffffffffu, mlo), whi = __reduce_or_sync(0xffffffffu, mhi);
+        while (wlo | whi) {
+          const int k = wlo ? __ffs(wlo) - 1 : 32 + __ffs(whi) - 1;
+          if (k < 32) wlo &= wlo - 1; else whi &= whi - 1;
+          uint32_t sbits = tmem_ld1(tS + k);
+          tmem_wait_dep1(sbits);
+          const bool mine = (k < 32 ? (mlo >> k) : (mhi >> (k - 32))) & 1u;
+          if (mine) {
+            const float u = pcode_f(__fmaf_rn(__uint_as_float(sbits), c18, -m), sTau);
+            sP[swz<64>(r, k)] = static_cast<uint8_t>(pack_e4m3x4(u, 0.f, 0.f, 0.f) & 0xFFu);
+          }
+        }
+      }
+      // keys past N in the last block take code 0
+      for (int k = nvalid; k < kBN; ++k) sP[swz<64>(r, k)] = 0;
+      if (DUMP) {
         for (int k = 0; k < kBN; ++k) {
           uint32_t sbits = tmem_ld1(tS + k);
           tmem_wait_dep1(sbits);
-          const float sk_ = __uint_as_float(sbits);
-          if (fix || k >= nvalid || DUMP) {
-            const float u = k < nvalid ? pcode_f(__fmaf_rn(sk_, c18, -m), sTau) : 0.f;
-            sP[swz<64>(r, k)] = static_cast<uint8_t>(pack_e4m3x4(u, 0.f, 0.f, 0.f) & 0xFFu);
-            if (DUMP && k < nvalid && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr) {
-              const size_t base = (size_t)(row - p.dbg_r0) * p.N + (size_t)j * kBN;
-              p.s_dump[base + k] = static_cast<int32_t>(sk_ * 262144.f);
-            }
-          }
+          if (k < nvalid && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr)
+            p.s_dump[(size_t)(row - p.dbg_r0) * p.N + (size_t)j * kBN + k] =
+                static_cast<int32_t>(__uint_as_float(sbits) * 262144.f);
         }
       }
       tc_fence_before();
@@ -546,6 +537,47 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }
+}
+
+// Widens the packed K / V codes of one (head, 64-key block) into the exact
+// shared-memory images of the attention kernel's operand tiles: K as 64 rows
+// x D e4m3 subnormals (K-major, 128B / 64B swizzle), V^T as D rows x 64 keys
+// (64B swizzle), followed by the block's V scales times 2^9.  HBM-bound.
+template <int D>
+__global__ void __launch_bounds__(256) widen_kv_kernel(const __grid_constant__ Int4Params p, uint8_t* work) {
+  using L = Int4Smem<D>;
+  const int j = blockIdx.x, h = p.heads[blockIdx.y], b = blockIdx.z;
+  const size_t head = (size_t)b * p.H + h;
+  const int npad = p.nblk * kBN;
+  uint8_t* img = work + (head * p.nblk + j) * (size_t)L::IMG_BYTES;
+  const uint8_t* kp = p.k_codes + (head * npad + (size_t)j * kBN) * (D / 2);
+  for (int i = threadIdx.x; i < kBN * D / 32; i += blockDim.x) {
+    const int rr = i / (D / 32), cg = i % (D / 32);
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(kp + 16 * i));
+    uint32_t o[8];
+    codes8_to_e4m3(w.x, o[0], o[1]);
+    codes8_to_e4m3(w.y, o[2], o[3]);
+    codes8_to_e4m3(w.z, o[4], o[5]);
+    codes8_to_e4m3(w.w, o[6], o[7]);
+    *reinterpret_cast<uint4*>(img + swz<L::ROWB>(rr, cg * 32)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(img + swz<L::ROWB>(rr, cg * 32 + 16)) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+  const uint8_t* vp = p.v_codes + (head * p.nblk + j) * (size_t)D * 32;
+  uint8_t* vimg = img + L::K_BYTES;
+  for (int i = threadIdx.x; i < D * 2; i += blockDim.x) {
+    const int c = i >> 1, hl = i & 1;
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(vp + 16 * i));
+    uint32_t o[8];
+    codes8_to_e4m3(w.x, o[0], o[1]);
+    codes8_to_e4m3(w.y, o[2], o[3]);
+    codes8_to_e4m3(w.z, o[4], o[5]);
+    codes8_to_e4m3(w.w, o[6], o[7]);
+    *reinterpret_cast<uint4*>(vimg + swz<64>(c, hl * 32)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(vimg + swz<64>(c, hl * 32 + 16)) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+  float* sv = reinterpret_cast<float*>(img + L::K_BYTES + L::VIMG_BYTES);
+  const float* vs = p.v_scale + (head * p.nblk + j) * D;
+  for (int c = threadIdx.x; c < D; c += blockDim.x) sv[c] = __ldg(vs + c) * 512.f;
 }
 
 // Exhaustive-check hook: the kernel's P-code function on an array.

@@ -157,6 +157,7 @@ rota_status rota_attn_buffer_sizes(const rota_attn_desc* d, size_t* bytes) {
   bytes[ROTA_BUF_ROPE_TABLE] = 4 * (static_cast<size_t>(d->grid_t) * (d->rope_dim[0] / 2) +
                                     static_cast<size_t>(d->grid_h) * (d->rope_dim[1] / 2) +
                                     static_cast<size_t>(d->grid_w) * (d->rope_dim[2] / 2));
+  bytes[ROTA_BUF_INT4_WORK] = heads * nblk * (D == 128 ? rota::Int4Smem<128>::IMG_BYTES : rota::Int4Smem<64>::IMG_BYTES);
   return ROTA_OK;
 }
 
@@ -249,7 +250,8 @@ static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers*
   rota_status st = rota_attn_validate(d);
   if (st != ROTA_OK) return st;
   if (!buf || !out || !aligned16(out)) return ROTA_ERR_INVALID_ARG;
-  const void* need[] = {buf->q_codes, buf->k_codes, buf->q_scale, buf->k_scale, buf->v_codes, buf->v_scale};
+  const void* need[] = {buf->q_codes, buf->k_codes, buf->q_scale, buf->k_scale, buf->v_codes, buf->v_scale,
+                        buf->int4_work};
   for (const void* ptr : need)
     if (!ptr || !aligned16(ptr)) return ROTA_ERR_INVALID_ARG;
 
@@ -263,6 +265,7 @@ static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers*
   p.k_scale = buf->k_scale;
   p.v_codes = buf->v_codes;
   p.v_scale = buf->v_scale;
+  p.work = buf->int4_work;
   p.out = out;
   p.H = d->H;
   p.N = d->N;
@@ -295,13 +298,22 @@ static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers*
     p.k_scale += hs * nblk;
     p.v_codes += hs * nblk * D * 32;
     p.v_scale += hs * nblk * D;
+    p.work += hs * nblk * (D == 128 ? rota::Int4Smem<128>::IMG_BYTES : rota::Int4Smem<64>::IMG_BYTES);
     p.out += hs * d->N * D;
   } else {
     p.nheads = select_heads(d, head_flags, 0, p.heads);
     if (p.nheads == 0) return ROTA_OK;
   }
-  const dim3 grid((d->N + rota::kRowsPerCta - 1) / rota::kRowsPerCta, p.nheads, batches);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // 1. widen the K / V codes of the selected heads once
+  const dim3 wgrid(p.nblk, p.nheads, batches);
+  if (d->head_dim == 128)
+    rota::widen_kv_kernel<128><<<wgrid, 256, 0, s>>>(p, const_cast<uint8_t*>(p.work));
+  else
+    rota::widen_kv_kernel<64><<<wgrid, 256, 0, s>>>(p, const_cast<uint8_t*>(p.work));
+  if ((st = cuda_status(cudaGetLastError())) != ROTA_OK) return st;
+  // 2. attention
+  const dim3 grid((d->N + rota::kRowsPerCta - 1) / rota::kRowsPerCta, p.nheads, batches);
   if (d->head_dim == 128)
     st = dump ? launch_int4_kernel(rota::attn_int4_kernel<128, true>, rota::Int4Smem<128>::ALLOC, grid, s, p)
               : launch_int4_kernel(rota::attn_int4_kernel<128, false>, rota::Int4Smem<128>::ALLOC, grid, s, p);
@@ -433,9 +445,10 @@ extern "C" rota_status rota_attn_fwd_int4_noalloc(const rota_attn_desc* d, const
   if ((st = rota_attn_buffer_sizes(d, sz)) != ROTA_OK) return st;
   const size_t table_floats = sz[ROTA_BUF_ROPE_TABLE] / 4;
   const int order[] = {ROTA_BUF_Q_CODES, ROTA_BUF_K_CODES, ROTA_BUF_Q_SCALE, ROTA_BUF_K_SCALE,
-                       ROTA_BUF_V_CODES, ROTA_BUF_V_SCALE, ROTA_BUF_ROPE_TABLE, ROTA_BUF_ROPE_TABLE};
-  size_t off[8], total = 0;
-  for (int i = 0; i < 8; ++i) {
+                       ROTA_BUF_V_CODES, ROTA_BUF_V_SCALE, ROTA_BUF_ROPE_TABLE, ROTA_BUF_ROPE_TABLE,
+                       ROTA_BUF_INT4_WORK};
+  size_t off[9], total = 0;
+  for (int i = 0; i < 9; ++i) {
     off[i] = total;
     total += round256(sz[order[i]]);
   }
@@ -466,6 +479,7 @@ extern "C" rota_status rota_attn_fwd_int4_noalloc(const rota_attn_desc* d, const
   b.v_scale = reinterpret_cast<float*>(s + off[5]);
   b.rope_cos = reinterpret_cast<const float*>(s + off[6]);
   b.rope_sin = reinterpret_cast<const float*>(s + off[7]);
+  b.int4_work = s + off[8];
   if ((st = rota_attn_prepare_qk(d, q, k, v, nullptr, &b, stream)) != ROTA_OK) return st;
   return rota_attn_fwd_int4(d, &b, nullptr, out, stream);
 }

@@ -24,7 +24,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 ROTA_OK, ROTA_ERR_INVALID_ARG, ROTA_ERR_UNSUPPORTED, ROTA_ERR_CUDA, ROTA_ERR_TIMEOUT, ROTA_ERR_DEVICE = range(6)
 (ROTA_BUF_Q_CODES, ROTA_BUF_K_CODES, ROTA_BUF_Q_SCALE, ROTA_BUF_K_SCALE, ROTA_BUF_V_CODES,
- ROTA_BUF_V_SCALE, ROTA_BUF_Q_ROPE, ROTA_BUF_K_ROPE, ROTA_BUF_ROPE_TABLE, ROTA_BUF_COUNT) = range(10)
+ ROTA_BUF_V_SCALE, ROTA_BUF_Q_ROPE, ROTA_BUF_K_ROPE, ROTA_BUF_ROPE_TABLE, ROTA_BUF_INT4_WORK,
+ ROTA_BUF_COUNT) = range(11)
 
 
 class rota_attn_desc(ctypes.Structure):
@@ -40,7 +41,8 @@ class rota_attn_buffers(ctypes.Structure):
                 ("q_scale", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
                 ("v_codes", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
                 ("q_rope", ctypes.c_void_p), ("k_rope", ctypes.c_void_p),
-                ("rope_cos", ctypes.c_void_p), ("rope_sin", ctypes.c_void_p)]
+                ("rope_cos", ctypes.c_void_p), ("rope_sin", ctypes.c_void_p),
+                ("int4_work", ctypes.c_void_p)]
 
 
 _P = ctypes.c_void_p
@@ -203,6 +205,7 @@ class RotaAttention:
         self.q_codes, self.k_codes = u8(sz[ROTA_BUF_Q_CODES]), u8(sz[ROTA_BUF_K_CODES])
         self.q_scale, self.k_scale = u8(sz[ROTA_BUF_Q_SCALE]), u8(sz[ROTA_BUF_K_SCALE])
         self.v_codes, self.v_scale = u8(sz[ROTA_BUF_V_CODES]), u8(sz[ROTA_BUF_V_SCALE])
+        self.int4_work = u8(sz[ROTA_BUF_INT4_WORK])
         self.q_rope = u8(sz[ROTA_BUF_Q_ROPE]) if need_fp16 else None
         self.k_rope = u8(sz[ROTA_BUF_K_ROPE]) if need_fp16 else None
         c, s = rota_attn_build_rope_tables(desc)
@@ -210,7 +213,7 @@ class RotaAttention:
         self.rope_sin = torch.from_numpy(s).to(self.device)
         b = rota_attn_buffers()
         for name in ("q_codes", "k_codes", "q_scale", "k_scale", "v_codes", "v_scale", "q_rope", "k_rope",
-                     "rope_cos", "rope_sin"):
+                     "rope_cos", "rope_sin", "int4_work"):
             setattr(b, name, _ptr(getattr(self, name)))
         self.buffers = b
 
