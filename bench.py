@@ -111,6 +111,17 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(values, pg, device=None):
+    """Element-wise max of a list of floats over all ranks (identity without a
+    process group).  The same collective runs on every rank, in the same order."""
+    if pg is None:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
 def workload_config(w, l2_note):
     return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} head_dim={w.d} RoPE "
                         f"{'/'.join(map(str, w.rope_dim))} grid {'x'.join(map(str, w.grid))} "
@@ -286,10 +297,7 @@ def main():
         raise RuntimeError(f"device error in the timed region: {ra.rota_attn_status_string(st)}")
 
     ms_step = ms_total / args.steps
-    if pg is not None:
-        tt = torch.tensor([ms_step, ms_e2e], dtype=torch.float64, device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        ms_step, ms_e2e = float(tt[0]), float(tt[1])
+    ms_step, ms_e2e = max_over_ranks([ms_step, ms_e2e], pg, dev)
 
     if rank == 0:
         ops = w.ops()
