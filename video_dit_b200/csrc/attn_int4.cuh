@@ -241,35 +241,38 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         // ---- MMA issuer ----
         constexpr uint32_t ID_S = idesc(1, 0, 0, kBM, kBN);      // e4m3 x e4m3 -> f32, 128 x 64
         constexpr uint32_t ID_PV = idesc(1, 0, 0, kBM, L::NPV);  // 128 x (D + 16)
-        const uint32_t qa0 = smem_u32(smem + L::OFF_Q), qa1 = qa0 + L::Q_BYTES;
-        const uint32_t pbase = smem_u32(smem + L::OFF_P);  // P buffer (tile t, block j) at (2t + (j & 1)) * P_BYTES
+        // descriptors: constant high words, low words stepped by 32 bytes (2 units) per K step
+        const uint32_t hi_qk = sdesc_hi(L::SBO_QK, L::LAYOUT_QK), hi_64 = sdesc_hi(512, 4);
+        const uint32_t lo_q0 = sdesc_lo(smem_u32(smem + L::OFF_Q)), lo_q1 = lo_q0 + (L::Q_BYTES >> 4);
+        const uint32_t lo_p = sdesc_lo(smem_u32(smem + L::OFF_P));   // + (2t + (j & 1)) * P_BYTES / 16
+        const uint32_t lo_op = sdesc_lo(smem_u32(smem + L::OFF_OP));  // + op * OP_BYTES / 16
         bool ok = mbar_wait(q_full, 0, lim);
         auto issue_s = [&](int j, int t) -> bool {
           const int op = j % kOps;
           if (!mbar_wait(&s_empty[t], (j & 1) ^ 1, lim)) return false;
           tc_fence_after();
           if (p.inject_skip && j == 0 && t == 0) return true;  // fault injection: never committed
-          const uint32_t ka = smem_u32(smem + L::OFF_OP + op * L::OP_BYTES);
-          const uint32_t qa = t ? qa1 : qa0;
+          const uint32_t lk = lo_op + op * (L::OP_BYTES >> 4);
+          const uint32_t lq = t ? lo_q1 : lo_q0;
+          const uint32_t d = tmem + (t ? L::T_S1 : L::T_S0);
+          mma_f8f6f4_lh<0>(d, lq, hi_qk, lk, hi_qk, ID_S);
 #pragma unroll
-          for (int k = 0; k < D / 32; ++k)
-            mma_f8f6f4(tmem + (t ? L::T_S1 : L::T_S0), sdesc(qa + 32 * k, L::SBO_QK, L::LAYOUT_QK),
-                       sdesc(ka + 32 * k, L::SBO_QK, L::LAYOUT_QK), ID_S, k > 0);
+          for (int k = 1; k < D / 32; ++k) mma_f8f6f4_lh<1>(d, lq + 2 * k, hi_qk, lk + 2 * k, hi_qk, ID_S);
           mma_commit(&s_full[t]);
           return true;
         };
         auto issue_pv = [&](int j) -> bool {
           const int op = j % kOps;
-          const uint32_t va = smem_u32(smem + L::OFF_OP + op * L::OP_BYTES + L::K_BYTES);
+          const uint32_t lv = lo_op + op * (L::OP_BYTES >> 4) + (L::K_BYTES >> 4);
           for (int t = 0; t < 2; ++t) {
             if (!mbar_wait(&p_full[2 * t + (j & 1)], (j >> 1) & 1, lim)) return false;
             if (!mbar_wait(&pv_empty[t], (j & 1) ^ 1, lim)) return false;
             tc_fence_after();
-            const uint32_t pa = pbase + (2 * t + (j & 1)) * L::P_BYTES;
+            const uint32_t lp = lo_p + (2 * t + (j & 1)) * (L::P_BYTES >> 4);
+            const uint32_t d = tmem + (t ? L::T_PV1 : L::T_PV0);
+            mma_f8f6f4_lh<0>(d, lp, hi_64, lv, hi_64, ID_PV);
 #pragma unroll
-            for (int k = 0; k < kBN / 32; ++k)
-              mma_f8f6f4(tmem + (t ? L::T_PV1 : L::T_PV0), sdesc(pa + 32 * k, 512, 4), sdesc(va + 32 * k, 512, 4),
-                         ID_PV, k > 0);
+            for (int k = 1; k < kBN / 32; ++k) mma_f8f6f4_lh<1>(d, lp + 2 * k, hi_64, lv + 2 * k, hi_64, ID_PV);
             mma_commit(&pv_full[t]);
           }
           mma_commit(&op_empty[op]);
