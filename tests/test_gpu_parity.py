@@ -21,6 +21,8 @@ CASES = {
     "wan_mini": synth.scaled(synth.WORKLOADS["wan480"], "wan_mini", H=3, grid=(3, 10, 13)),     # N=390
     "hunyuan_mini": synth.scaled(synth.WORKLOADS["hunyuan"], "hy_mini", H=2, grid=(3, 9, 20)),  # N=540
     "ragged_small": synth.scaled(synth.WORKLOADS["wan480"], "ragged", H=1, grid=(1, 3, 7)),     # N=21 < 64
+    # uneven RoPE split: rotation blocks start at channels 42 and 86, off any power-of-two grid
+    "offgrid": synth.scaled(synth.WORKLOADS["wan480"], "offgrid", H=2, grid=(2, 7, 11), rope_dim=(42, 44, 42)),
 }
 
 # Many key blocks per CTA (74), so every pipeline stage and barrier phase wraps many times.
