@@ -23,6 +23,8 @@ CASES = {
     "ragged_small": synth.scaled(synth.WORKLOADS["wan480"], "ragged", H=1, grid=(1, 3, 7)),     # N=21 < 64
     # uneven RoPE split: rotation blocks start at channels 42 and 86, off any power-of-two grid
     "offgrid": synth.scaled(synth.WORKLOADS["wan480"], "offgrid", H=2, grid=(2, 7, 11), rope_dim=(42, 44, 42)),
+    # rotation blocks of 32 and 64 channels (the largest Hadamard orders)
+    "wide_blocks": synth.scaled(synth.WORKLOADS["wan480"], "wide", H=1, grid=(2, 5, 7), rope_dim=(32, 32, 64)),
 }
 
 # Many key blocks per CTA (74), so every pipeline stage and barrier phase wraps many times.

@@ -100,6 +100,31 @@ __device__ __forceinline__ float rope_rotate_unit(float* xrow, int c0, int pair0
   return amax;
 }
 
+// The same unit for G >= 16, in place in the smem row (no register arrays).
+__device__ __noinline__ float rope_rotate_unit_smem(float* xrow, int c0, int G, int pair0, const float* ct,
+                                                   const float* st, bool rot, float rnorm) {
+  float* y = xrow + c0;
+  for (int j = 0; j < G / 2; ++j) {
+    float x0 = y[2 * j], x1 = y[2 * j + 1];
+    rope_pair(x0, x1, __ldg(ct + pair0 + j), __ldg(st + pair0 + j));
+    y[2 * j] = x0;
+    y[2 * j + 1] = x1;
+  }
+  if (rot) {
+    for (int h = 1; h < G; h <<= 1)
+      for (int j = 0; j < G; ++j) {
+        if (j & h) continue;
+        const float u = y[j], w = y[j + h];
+        y[j] = __fadd_rn(u, w);
+        y[j + h] = __fsub_rn(u, w);
+      }
+    for (int j = 0; j < G; ++j) y[j] = __fmul_rn(y[j], rnorm);
+  }
+  float amax = 0.f;
+  for (int j = 0; j < G; ++j) amax = fmaxf(amax, fabsf(y[j]));
+  return amax;
+}
+
 __device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -133,33 +158,37 @@ __device__ __forceinline__ uint32_t pack8(const int (&c)[8]) {
 }
 
 // fp16 tile [64, D] of one (head, block) -> fp32 smem rows of stride D+1.
+// Every thread issues all of its 16-byte loads before it converts any, so a
+// CTA waits for one memory latency rather than one per load.
 template <int D>
 __device__ __forceinline__ void load_tile(const __half* src, int n0, int N, float* X) {
   constexpr int LD = D + 1;
-  for (int i = threadIdx.x; i < 64 * D / 8; i += kPrologueThreads) {
+  constexpr int PER = 64 * D / 8 / kPrologueThreads;
+  static_assert(PER * kPrologueThreads * 8 == 64 * D, "tile split");
+  uint4 u[PER];
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int i = threadIdx.x + k * kPrologueThreads;
     const int r = i / (D / 8), ch = i % (D / 8);
     const int n = n0 + r;
-    float f[8];
-    if (n < N) {
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + (size_t)n * D + ch * 8));
-      const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+    u[k] = n < N ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)n * D + ch * 8)) : make_uint4(0, 0, 0, 0);
+  }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 t = __half22float2(h2[j]);
-        f[2 * j] = t.x;
-        f[2 * j + 1] = t.y;
-      }
-    } else {
+  for (int k = 0; k < PER; ++k) {
+    const int i = threadIdx.x + k * kPrologueThreads;
+    const int r = i / (D / 8), ch = i % (D / 8);
+    const __half2* h2 = reinterpret_cast<const __half2*>(&u[k]);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) f[j] = 0.f;
+    for (int j = 0; j < 4; ++j) {
+      const float2 t = __half22float2(h2[j]);
+      X[r * LD + ch * 8 + 2 * j] = t.x;
+      X[r * LD + ch * 8 + 2 * j + 1] = t.y;
     }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) X[r * LD + ch * 8 + j] = f[j];
   }
 }
 
 template <int D>
-__global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(const PrologueParams p) {
+__global__ void __launch_bounds__(kPrologueThreads, 4) prologue_kernel(const PrologueParams p) {
   constexpr int LD = D + 1;
   __shared__ float X[64 * LD];
   __shared__ float red[kPrologueThreads / 32];
@@ -232,9 +261,7 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(const Prolog
           case 2: m = rope_rotate_unit<2>(xrow, c0, pair0, ct, st, rot, p.rnorm[a]); break;
           case 4: m = rope_rotate_unit<4>(xrow, c0, pair0, ct, st, rot, p.rnorm[a]); break;
           case 8: m = rope_rotate_unit<8>(xrow, c0, pair0, ct, st, rot, p.rnorm[a]); break;
-          case 16: m = rope_rotate_unit<16>(xrow, c0, pair0, ct, st, rot, p.rnorm[a]); break;
-          case 32: m = rope_rotate_unit<32>(xrow, c0, pair0, ct, st, rot, p.rnorm[a]); break;
-          default: m = rope_rotate_unit<64>(xrow, c0, pair0, ct, st, rot, p.rnorm[a]); break;
+          default: m = rope_rotate_unit_smem(xrow, c0, G, pair0, ct, st, rot, p.rnorm[a]); break;
         }
         amax = fmaxf(amax, m);
       }
@@ -268,26 +295,36 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(const Prolog
   if (flagged) return;
   load_tile<D>(p.v + head * p.N * D, n0, p.N, X);
   __syncthreads();
-  for (int c = threadIdx.x; c < D; c += kPrologueThreads) {
+  // kPrologueThreads / D neighbouring lanes share a channel, each taking 64 / TPC rows
+  constexpr int TPC = kPrologueThreads / D;
+  constexpr int RPT = 64 / TPC;
+  static_assert(TPC * D == kPrologueThreads && RPT % 8 == 0, "V split");
+  {
+    const int c = threadIdx.x / TPC, part = threadIdx.x % TPC;
+    const int r0 = part * RPT;
     float amax = 0.f;
-    for (int r = 0; r < 64; ++r) amax = fmaxf(amax, fabsf(X[r * LD + c]));
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) amax = fmaxf(amax, fabsf(X[(r0 + r) * LD + c]));
+#pragma unroll
+    for (int o = 1; o < TPC; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float scale = amax == 0.f ? 0.f : __fdiv_rn(amax, 7.f);
     const float inv = amax == 0.f ? 0.f : __fdiv_rn(7.f, amax);
-    uint32_t w[8];
+    uint32_t w[RPT / 8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < RPT / 8; ++j) {
       int cs[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        const int r = 8 * j + t;
+        const int r = r0 + 8 * j + t;
         cs[t] = (n0 + r < p.N) ? quant_code(X[r * LD + c], inv) : 0;
       }
       w[j] = pack8(cs);
     }
-    uint4* dst = reinterpret_cast<uint4*>(p.v_codes + ((head * p.nblk + blk) * D + c) * 32);
-    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    p.v_scale[(head * p.nblk + blk) * D + c] = scale;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(p.v_codes + ((head * p.nblk + blk) * D + c) * 32) + part * (RPT / 8);
+#pragma unroll
+    for (int j = 0; j < RPT / 8; j += 4)
+      *reinterpret_cast<uint4*>(dst + j) = make_uint4(w[j], w[j + 1], w[j + 2], w[j + 3]);
+    if (part == 0) p.v_scale[(head * p.nblk + blk) * D + c] = scale;
   }
 }
 
