@@ -1,16 +1,29 @@
 // attn_fp16.cuh -- FP16 FlashAttention forward for the flagged heads.
 //
 // "RotateAttention: RoPE-Aware Rotation and Range Rectification for INT4
-// Quantized Attention in Video Generation", abstract: "selective FP16
-// fallback for accuracy-sensitive attention blocks and denoising steps".
+// Quantized Attention in Video Generation", abstract: selective FP16 fallback
+// for accuracy-sensitive attention blocks and denoising steps.  A flagged
+// head is plain softmax attention over the RoPE'd fp16 Q, K and the fp16 V:
+// fp32 scores, fp32 exponentials, P rounded to fp16 for the P V product, fp32
+// accumulation.
 //
-// Per CTA: 128 query rows of one flagged head, thread i owns row i.
-// Per 64-key block: fp16 K (K-major) and V^T tiles staged in shared memory,
-// S = Q K^T on the tensor core (tcgen05.mma kind::f16, fp32 in TMEM), an fp32
-// online softmax in base 2, P rounded to fp16 into shared memory, acc = P V
-// (kind::f16, fp32 in TMEM), O = O * alpha + acc in registers; out = O / l.
+// One CTA = two 128-row query tiles of one flagged head, 384 threads:
+//   warp 0      TMA producer: the two Q tiles once, then the K and V tiles of
+//               each 64-key block (tensor-map loads straight from q_rope,
+//               k_rope and v, 128-byte swizzle) into a 3-stage ring;
+//   warp 1      TMEM owner and MMA issuer (one thread);
+//   warps 2-3   idle;
+//   warps 4-7   tile 0, warps 8-11 tile 1 (thread = row = TMEM lane).
+// S_t(j) = Q_t K_j^T (kind::f16, fp32 in TMEM, two buffers per tile).  O_t
+// accumulates in TMEM across blocks: the MMA adds P_t(j) V_j to it, where V_j
+// is read as it sits in memory (channels contiguous: an MN-major B operand).
+// The exponentials use a reference max m_ref per row that is raised only when
+// a block's max exceeds it by more than 8 (log2 units): P stays <= 2^8, which
+// fp16 holds, and O and l are rescaled in place only then (a warp rescales
+// its TMEM rows after the previous P V has landed).  out = O / l.
 #pragma once
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_fp16.h>
 
 #include "sm100.cuh"
@@ -18,9 +31,9 @@
 namespace rota {
 
 struct Fp16Params {
-  const __half* q_rope;
-  const __half* k_rope;
-  const __half* v;
+  CUtensorMap tm_q;   // q_rope as [B*H*N rows, D] fp16, box 64 x 128 rows
+  CUtensorMap tm_k;   // k_rope, box 64 x 64 rows
+  CUtensorMap tm_v;   // v,      box 64 x 64 rows
   float* out;
   int H, N;
   float scale_log2;     // RN(sm_scale * log2 e)
@@ -29,202 +42,297 @@ struct Fp16Params {
   int16_t heads[256];
 };
 
-constexpr int kF16Threads = 128;
+constexpr int kF16Threads = 384;
+constexpr int kF16Stages = 3;
+constexpr float kRescaleLog2 = 8.f;   // raise the reference max only past this margin
 
 template <int D>
 struct F16Smem {
-  static constexpr int KATOMS = D * 2 / 128;      // 128-byte K atoms per Q/K row
-  static constexpr int Q_BYTES = kBM * D * 2;
-  static constexpr int K_BYTES = kBN * D * 2;
-  static constexpr int V_BYTES = D * kBN * 2;     // V^T: D rows of 64 keys (128 B)
-  static constexpr int P_BYTES = kBM * kBN * 2;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + K_BYTES;
-  static constexpr int OFF_P = OFF_V + V_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
-  static constexpr int OFF_TMEM = OFF_BAR + 8;
-  static constexpr int OFF_FLAG = OFF_TMEM + 4;
-  static constexpr int BYTES = OFF_FLAG + 4;
+  static constexpr int ATOMS = D / 64;                 // 128-byte (64-channel) column atoms
+  static constexpr int Q_BYTES = kBM * D * 2;          // one tile: ATOMS x [128 rows x 128 B]
+  static constexpr int K_BYTES = kBN * D * 2;          // ATOMS x [64 keys x 128 B], K-major
+  static constexpr int V_BYTES = kBN * D * 2;          // ATOMS x [64 keys x 128 B], channels contiguous
+  static constexpr int STAGE_BYTES = K_BYTES + V_BYTES;
+  static constexpr int P_BYTES = kBM * kBN * 2;        // [128 rows x 128 B]
+  static constexpr int OFF_Q = 0;                                // 2 tiles
+  static constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;             // kF16Stages stages
+  static constexpr int OFF_P = OFF_KV + kF16Stages * STAGE_BYTES;  // 2 tiles x 2 buffers
+  static constexpr int OFF_BAR = OFF_P + 4 * P_BYTES;
+  // barriers: kv_full[3] kv_empty[3] s_full[4] s_empty[4] p_full[4] p_empty[4]
+  //           o_ready[2] q_full mma_done
+  static constexpr int NBAR = 3 + 3 + 4 + 4 + 4 + 4 + 2 + 1 + 1;
+  static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_ABORT = OFF_TMEM + 4;
+  static constexpr int BYTES = OFF_ABORT + 4;
   static constexpr int ALLOC = BYTES + 1024;
-  static constexpr int TMEM_COLS = (kBN + D) <= 128 ? 128 : 256;
+  static constexpr uint32_t TMEM_COLS = 512;
+  // S of tile t, buffer b at column (2t + b) * 64; O of tile t at 256 + t * D
+  static constexpr uint32_t T_S = 0, T_O = 4 * kBN;
+  static_assert(T_O + 2 * D <= TMEM_COLS, "TMEM budget");
+  static_assert(ALLOC <= 232448, "shared memory budget");
+  static_assert(Q_BYTES % 1024 == 0 && K_BYTES % 1024 == 0 && P_BYTES % 1024 == 0, "swizzle atom alignment");
 };
-
-// Byte offset of (row, byte k) in a K-major fp16 tile of `rows` rows stored as
-// consecutive [rows x 128 B] atoms along K, 128-byte swizzle.
-__device__ __forceinline__ uint32_t swz_atoms(uint32_t row, uint32_t kbyte, uint32_t rows) {
-  return (kbyte >> 7) * rows * 128 + swz<128>(row, kbyte & 127);
-}
 
 template <int D>
 __global__ void __launch_bounds__(kF16Threads, 1) attn_fp16_kernel(const __grid_constant__ Fp16Params p) {
   using L = F16Smem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem + L::OFF_Q;
-  uint8_t* sK = smem + L::OFF_K;
-  uint8_t* sV = smem + L::OFF_V;
-  uint8_t* sP = smem + L::OFF_P;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + 3;
+  // per (tile t, buffer b) = index 2t + b, buffer b = block parity: each
+  // completes once per use of its buffer (phase (j >> 1) & 1 for block j)
+  uint64_t* s_full = bars + 6;
+  uint64_t* s_empty = bars + 10;
+  uint64_t* p_full = bars + 14;
+  uint64_t* p_empty = bars + 18;   // the P V that read P buffer 2t + b has completed
+  uint64_t* o_ready = bars + 22;   // P_t(j) V_j has completed (once per block)
+  uint64_t* q_full = bars + 24;
+  uint64_t* mma_done = bars + 25;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
-  int* sAbort = reinterpret_cast<int*>(smem + L::OFF_FLAG);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(smem + L::OFF_ABORT);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int qt = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = p.heads[blockIdx.y];
   const int b = blockIdx.z;
   const size_t head = (size_t)b * p.H + h;
-  const int row = qt * kBM + tid;
+  const int row_base = (int)(head * p.N);           // first row of this head in the [B*H*N, D] views
+  const int q0 = blockIdx.x * (2 * kBM);
   const int nkb = (p.N + kBN - 1) / kBN;
+  const uint64_t lim = p.timeout_ns;
 
   if (tid == 0) {
-    mbar_init(bar, 1);
-    fence_mbar_init();
+    for (int i = 0; i < kF16Stages; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&p_empty[i], 1);
+    }
+    mbar_init(&o_ready[0], 1);
+    mbar_init(&o_ready[1], 1);
+    mbar_init(q_full, 1);
+    mbar_init(mma_done, 1);
     *sAbort = 0;
+    fence_mbar_init();
   }
   __syncwarp();
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(sTmem, L::TMEM_COLS);
     tmem_relinquish();
-  }
-  {
-    const __half* qsrc = p.q_rope + head * p.N * D;
-    for (int i = tid; i < kBM * D / 8; i += kF16Threads) {
-      const int r = i / (D / 8), c = i % (D / 8);
-      const int n = qt * kBM + r;
-      uint4 w = make_uint4(0, 0, 0, 0);
-      if (n < p.N) w = __ldg(reinterpret_cast<const uint4*>(qsrc + (size_t)n * D + c * 8));
-      *reinterpret_cast<uint4*>(sQ + swz_atoms(r, c * 16, kBM)) = w;
-    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sTmem;
-  const uint32_t t_lane = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t tS = tmem, tO = tmem + kBN;
-  constexpr uint32_t ID_S = idesc(1, 0, 0, kBM, kBN);   // f16 x f16 -> f32
-  constexpr uint32_t ID_PV = idesc(1, 0, 0, kBM, D);
 
-  float O[D];
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- TMA producer ----
+      mbar_arrive_expect_tx(q_full, 2 * L::Q_BYTES);
+      for (int t = 0; t < 2; ++t)
+        for (int a = 0; a < L::ATOMS; ++a)
+          tma_load_2d(smem + L::OFF_Q + t * L::Q_BYTES + a * (kBM * 128), &p.tm_q, 64 * a, row_base + q0 + t * kBM,
+                      q_full);
+      int issued = 0;
+      for (int j = 0; j < nkb; ++j) {
+        const int st = j % kF16Stages;
+        if (!mbar_wait(&kv_empty[st], ((j / kF16Stages) & 1) ^ 1, lim)) { *sAbort = 1; break; }
+        if (*sAbort) break;
+        uint8_t* kt = smem + L::OFF_KV + st * L::STAGE_BYTES;
+        mbar_arrive_expect_tx(&kv_full[st], L::STAGE_BYTES);
+        for (int a = 0; a < L::ATOMS; ++a) {
+          tma_load_2d(kt + a * (kBN * 128), &p.tm_k, 64 * a, row_base + j * kBN, &kv_full[st]);
+          tma_load_2d(kt + L::K_BYTES + a * (kBN * 128), &p.tm_v, 64 * a, row_base + j * kBN, &kv_full[st]);
+        }
+        issued = j + 1;
+      }
+      // drain: every issued copy has landed before the CTA may exit
+      mbar_wait(q_full, 0, lim);
+      for (int j = (issued > kF16Stages ? issued - kF16Stages : 0); j < issued; ++j)
+        mbar_wait(&kv_full[j % kF16Stages], (j / kF16Stages) & 1, lim);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issuer ----
+      constexpr uint32_t ID_S = idesc(1, 0, 0, kBM, kBN);     // f16 x f16 -> f32, 128 x 64
+      constexpr uint32_t ID_PV = idesc(1, 0, 0, kBM, D, 1);   // B (V) channels-contiguous
+      const uint32_t q_addr = smem_u32(smem + L::OFF_Q), kv_addr = smem_u32(smem + L::OFF_KV);
+      const uint32_t p_addr = smem_u32(smem + L::OFF_P);
+      bool ok = mbar_wait(q_full, 0, lim);
+      auto issue_s = [&](int j, int t) -> bool {
+        const int sb = 2 * t + (j & 1);
+        if (!mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1, lim)) return false;
+        tc_fence_after();
+        const uint32_t qa = q_addr + t * L::Q_BYTES, ka = kv_addr + (j % kF16Stages) * L::STAGE_BYTES;
+        const uint32_t d = tmem + L::T_S + sb * kBN;
 #pragma unroll
-  for (int c = 0; c < D; ++c) O[c] = 0.f;
-  float m = -INFINITY, l = 0.f;
-  uint32_t phase = 0;
-  bool aborted = false;
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t atom = k >> 2, within = (k & 3) * 32;
+          mma_f16(d, sdesc(qa + atom * (kBM * 128) + within, 1024, 2), sdesc(ka + atom * (kBN * 128) + within, 1024, 2),
+                  ID_S, k > 0);
+        }
+        mma_commit(&s_full[sb]);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const uint32_t va = kv_addr + (j % kF16Stages) * L::STAGE_BYTES + L::K_BYTES;
+        for (int t = 0; t < 2; ++t) {
+          const int pb = 2 * t + (j & 1);
+          if (!mbar_wait(&p_full[pb], (j >> 1) & 1, lim)) return false;
+          tc_fence_after();
+          const uint32_t pa = p_addr + pb * L::P_BYTES;
+          const uint32_t d = tmem + L::T_O + t * D;
+#pragma unroll
+          for (int k = 0; k < kBN / 16; ++k)
+            mma_f16(d, sdesc(pa + 32 * k, 1024, 2), sdesc_lbo(va + 2048 * k, kBN * 128, 1024, 2), ID_PV,
+                    (j > 0 || k > 0) ? 1u : 0u);
+          mma_commit(&o_ready[t]);
+          mma_commit(&p_empty[pb]);
+        }
+        mma_commit(&kv_empty[j % kF16Stages]);
+        return true;
+      };
+      for (int j = 0; ok && j < nkb; ++j) {
+        if (!mbar_wait(&kv_full[j % kF16Stages], (j / kF16Stages) & 1, lim)) { ok = false; break; }
+        tc_fence_after();
+        if (!issue_s(j, 0) || !issue_s(j, 1)) { ok = false; break; }
+        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+        if (*sAbort) { ok = false; break; }
+      }
+      if (ok) ok = issue_pv(nkb - 1);
+      if (!ok) *sAbort = 1;
+      // every issued MMA completes before TMEM is released
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, lim);
+    }
+  } else if (warp >= 4) {
+    // ===================================================== query-tile warps
+    const int t = (warp - 4) >> 2;       // tile 0 or 1
+    const int r = tid & 127;             // row within the tile = TMEM lane
+    const int row = q0 + t * kBM + r;
+    const uint32_t t_lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS0 = tmem + L::T_S + 2 * t * kBN + t_lane;   // + (j & 1) * kBN
+    const uint32_t tO = tmem + L::T_O + t * D + t_lane;
+    const float c = p.scale_log2;
+    float m_ref = -INFINITY, l = 0.f;
+    bool aborted = false;
 
+    for (int j = 0; j < nkb; ++j) {
+      const int sb = 2 * t + (j & 1);
+      const uint32_t tS = tS0 + (j & 1) * kBN;
+      const int nvalid = min(kBN, p.N - j * kBN);
+      if (!warp_wait(&s_full[sb], (j >> 1) & 1, lim)) { aborted = true; break; }
+      tc_fence_after();
+      uint32_t sr[kBN];
+      {
+        uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+        uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+        tmem_ld32(tS, s0);
+        tmem_ld32(tS + 32, s1);
+        tmem_wait_dep2(s0, s1);
+      }
+      // S is in registers: the MMA may overwrite this buffer with S(j+2)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[sb]);
+      if (nvalid < kBN) {
+#pragma unroll
+        for (int k = 0; k < kBN; ++k)
+          if (k >= nvalid) sr[k] = __float_as_uint(-INFINITY);
+      }
+      float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < kBN; k += 8) {
+        x0 = max3(x0, __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
+        x1 = max3(x1, __uint_as_float(sr[k + 2]), __uint_as_float(sr[k + 3]));
+        x2 = max3(x2, __uint_as_float(sr[k + 4]), __uint_as_float(sr[k + 5]));
+        x3 = max3(x3, __uint_as_float(sr[k + 6]), __uint_as_float(sr[k + 7]));
+      }
+      const float m_blk = __fmul_rn(fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)), c);
+
+      // ---- raise the reference max (rare): rescale O (TMEM) and l ----
+      if (__any_sync(0xffffffffu, m_blk > m_ref + kRescaleLog2)) {
+        const float m_new = fmaxf(m_ref, m_blk);
+        const float alpha = ex2_approx(m_ref - m_new);   // 0 while O is empty (m_ref = -inf)
+        m_ref = m_new;
+        l *= alpha;
+        if (j > 0) {
+          // the previous block's P V has landed in O
+          if (!warp_wait(&o_ready[t], (j - 1) & 1, lim)) { aborted = true; break; }
+          tc_fence_after();
 #pragma unroll 1
-  for (int kb = 0; kb < nkb; ++kb) {
-    const __half* ksrc = p.k_rope + (head * p.N + (size_t)kb * kBN) * D;
-    const __half* vsrc = p.v + (head * p.N + (size_t)kb * kBN) * D;
-    const int nvalid = min(kBN, p.N - kb * kBN);
-    for (int i = tid; i < kBN * D / 8; i += kF16Threads) {
-      const int r = i / (D / 8), c = i % (D / 8);
-      uint4 kw = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
-      if (r < nvalid) {
-        kw = __ldg(reinterpret_cast<const uint4*>(ksrc + (size_t)r * D + c * 8));
-        vw = __ldg(reinterpret_cast<const uint4*>(vsrc + (size_t)r * D + c * 8));
-      }
-      *reinterpret_cast<uint4*>(sK + swz_atoms(r, c * 16, kBN)) = kw;
-      // V^T: channel rows of 64 keys; key r -> byte 2r of rows 8c .. 8c+7
-      const uint16_t* vh = reinterpret_cast<const uint16_t*>(&vw);
+          for (int cb = 0; cb < D / 32; ++cb) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * cb, o);
+            tmem_wait_dep(o);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) *reinterpret_cast<uint16_t*>(sV + swz<128>(c * 8 + j, 2 * r)) = vh[j];
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st32(tO + 32 * cb, o);
+          }
+          tmem_st_wait();
+        }
+      }
 
-    if (tid == 0) {
+      // ---- P = 2^(S c - m_ref) in fp16, row sum of the fp16 values in fp32 ----
+      uint32_t pw[kBN / 2];
+      float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+      for (int k = 0; k < kBN; k += 2) {
+        float d0, d1;
+        fma2(d0, d1, __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]), c, c, -m_ref, -m_ref);
+        const __half2 hp = __floats2half2_rn(ex2_approx(d0), ex2_approx(d1));
+        // l sums the fp16 values the P V product uses, so out = O / l is exact
+        // for a row whose weight sits on one key
+        const float2 back = __half22float2(hp);
+        add2(ls0, ls1, ls0, ls1, back.x, back.y);
+        pw[k / 2] = *reinterpret_cast<const uint32_t*>(&hp);
+      }
+      l += ls0 + ls1;
+      // the P V that read this buffer (block j - 2) has completed
+      if (j >= 2 && !warp_wait(&p_empty[sb], ((j >> 1) & 1) ^ 1, lim)) { aborted = true; break; }
+      uint8_t* sP = smem + L::OFF_P + sb * L::P_BYTES;
+#pragma unroll
+      for (int k = 0; k < kBN / 8; ++k)
+        *reinterpret_cast<uint4*>(sP + swz<128>(r, 16 * k)) =
+            make_uint4(pw[4 * k], pw[4 * k + 1], pw[4 * k + 2], pw[4 * k + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[sb]);
+      if (warp_flag(sAbort)) { aborted = true; break; }
+    }
+    // ---- epilogue: out = O / l once the last P V has landed ----
+    if (!aborted && !warp_wait(&o_ready[t], (nkb - 1) & 1, lim)) aborted = true;
+    if (aborted) {
+      *sAbort = 1;
+    } else {
       tc_fence_after();
-      const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK);
+      const float inv_l = 1.f / l;
+      float* dst = p.out + ((size_t)row_base + row) * D;
+#pragma unroll 1
+      for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * cb, o);
+        tmem_wait_dep(o);
+        if (row < p.N) {
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t atom = (k * 32) >> 7, within = (k * 32) & 127;
-        mma_f16(tS, sdesc(qa + atom * kBM * 128 + within, 1024, 2), sdesc(ka + atom * kBN * 128 + within, 1024, 2),
-                ID_S, k > 0);
-      }
-      mma_commit(bar);
-    }
-    if (!mbar_wait(bar, phase, p.timeout_ns)) *sAbort = 1;
-    phase ^= 1;
-    __syncthreads();
-    if (*sAbort) { aborted = true; break; }
-    tc_fence_after();
-
-    float s[kBN];
-    {
-      uint32_t r0[32], r1[32];
-      tmem_ld32(tS + t_lane, r0);
-      tmem_ld32(tS + t_lane + 32, r1);
-      tmem_wait_dep2(r0, r1);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        s[j] = __uint_as_float(r0[j]) * p.scale_log2;
-        s[32 + j] = __uint_as_float(r1[j]) * p.scale_log2;
+          for (int k = 0; k < 32; k += 4)
+            *reinterpret_cast<float4*>(dst + 32 * cb + k) =
+                make_float4(__uint_as_float(o[k]) * inv_l, __uint_as_float(o[k + 1]) * inv_l,
+                            __uint_as_float(o[k + 2]) * inv_l, __uint_as_float(o[k + 3]) * inv_l);
+        }
       }
     }
-    float bmax = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < kBN; ++j)
-      if (j < nvalid) bmax = fmaxf(bmax, s[j]);
-    const float m_new = fmaxf(m, bmax);
-    const float alpha = ex2_approx(m - m_new);
-    m = m_new;
-    float psum = 0.f;
-    uint32_t pw[kBN / 2];
-#pragma unroll
-    for (int j2 = 0; j2 < kBN / 2; ++j2) {
-      float p0 = (2 * j2 < nvalid) ? ex2_approx(s[2 * j2] - m) : 0.f;
-      float p1 = (2 * j2 + 1 < nvalid) ? ex2_approx(s[2 * j2 + 1] - m) : 0.f;
-      const __half2 hp = __floats2half2_rn(p0, p1);
-      const float2 back = __half22float2(hp);
-      psum += back.x + back.y;
-      pw[j2] = *reinterpret_cast<const uint32_t*>(&hp);
-    }
-    l = l * alpha + psum;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      *reinterpret_cast<uint4*>(sP + swz<128>(tid, 16 * j)) = make_uint4(pw[4 * j], pw[4 * j + 1], pw[4 * j + 2], pw[4 * j + 3]);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t pa = smem_u32(sP), va = smem_u32(sV);
-#pragma unroll
-      for (int k = 0; k < kBN / 16; ++k)
-        mma_f16(tO, sdesc(pa + 32 * k, 1024, 2), sdesc(va + 32 * k, 1024, 2), ID_PV, k > 0);
-      mma_commit(bar);
-    }
-    if (!mbar_wait(bar, phase, p.timeout_ns)) *sAbort = 1;
-    phase ^= 1;
-    __syncthreads();
-    if (*sAbort) { aborted = true; break; }
-    tc_fence_after();
-#pragma unroll
-    for (int j = 0; j < D / 32; ++j) {
-      uint32_t a[32];
-      tmem_ld32(tO + t_lane + 32 * j, a);
-      tmem_wait_dep(a);
-#pragma unroll
-      for (int t = 0; t < 32; ++t) O[32 * j + t] = __fmaf_rn(O[32 * j + t], alpha, __uint_as_float(a[t]));
-    }
-    tc_fence_before();
-    __syncthreads();
   }
 
-  if (!aborted && row < p.N) {
-    const float inv_l = 1.f / l;
-    float4* dst = reinterpret_cast<float4*>(p.out + (head * p.N + row) * D);
-#pragma unroll
-    for (int c4 = 0; c4 < D / 4; ++c4)
-      dst[c4] = make_float4(O[4 * c4] * inv_l, O[4 * c4 + 1] * inv_l, O[4 * c4 + 2] * inv_l, O[4 * c4 + 3] * inv_l);
-  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }

@@ -104,6 +104,53 @@ rota_status launch_int4_kernel(K kernel, int smem, dim3 grid, cudaStream_t s, co
 
 }  // namespace
 
+namespace {
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// [rows, D] fp16 tensor, boxes of 64 channels x box_rows rows, 128-byte swizzle.
+rota_status make_fp16_map(CUtensorMap* m, const void* base, uint64_t rows, int D, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return ROTA_ERR_CUDA;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ROTA_OK : ROTA_ERR_CUDA;
+}
+
+template <int D>
+rota_status launch_fp16_kernel(const rota::Fp16Params& p, dim3 grid, cudaStream_t s) {
+  using L = rota::F16Smem<D>;
+  rota_status st = set_smem(rota::attn_fp16_kernel<D>, L::ALLOC);
+  if (st != ROTA_OK) return st;
+  rota::attn_fp16_kernel<D><<<grid, rota::kF16Threads, L::ALLOC, s>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* rota_attn_status_string(rota_status s) {
@@ -346,26 +393,18 @@ rota_status rota_attn_fwd_fp16_fallback(const rota_attn_desc* d, const rota_attn
   p.nheads = select_heads(d, head_flags, 1, p.heads);
   if (p.nheads == 0) return ROTA_OK;
   if (!buf->q_rope || !buf->k_rope || !aligned16(buf->q_rope) || !aligned16(buf->k_rope)) return ROTA_ERR_INVALID_ARG;
-  p.q_rope = reinterpret_cast<const __half*>(buf->q_rope);
-  p.k_rope = reinterpret_cast<const __half*>(buf->k_rope);
-  p.v = reinterpret_cast<const __half*>(v);
+  const uint64_t rows = static_cast<uint64_t>(d->B) * d->H * d->N;
+  if ((st = make_fp16_map(&p.tm_q, buf->q_rope, rows, d->head_dim, rota::kBM)) != ROTA_OK) return st;
+  if ((st = make_fp16_map(&p.tm_k, buf->k_rope, rows, d->head_dim, rota::kBN)) != ROTA_OK) return st;
+  if ((st = make_fp16_map(&p.tm_v, v, rows, d->head_dim, rota::kBN)) != ROTA_OK) return st;
   p.out = out;
   p.H = d->H;
   p.N = d->N;
   p.scale_log2 = kappa_of(d);
   p.timeout_ns = kDefaultTimeoutNs;
-  const dim3 grid((d->N + rota::kBM - 1) / rota::kBM, p.nheads, d->B);
+  const dim3 grid((d->N + 2 * rota::kBM - 1) / (2 * rota::kBM), p.nheads, d->B);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d->head_dim == 128) {
-    using L = rota::F16Smem<128>;
-    if ((st = set_smem(rota::attn_fp16_kernel<128>, L::ALLOC)) != ROTA_OK) return st;
-    rota::attn_fp16_kernel<128><<<grid, rota::kF16Threads, L::ALLOC, s>>>(p);
-  } else {
-    using L = rota::F16Smem<64>;
-    if ((st = set_smem(rota::attn_fp16_kernel<64>, L::ALLOC)) != ROTA_OK) return st;
-    rota::attn_fp16_kernel<64><<<grid, rota::kF16Threads, L::ALLOC, s>>>(p);
-  }
-  return cuda_status(cudaGetLastError());
+  return d->head_dim == 128 ? launch_fp16_kernel<128>(p, grid, s) : launch_fp16_kernel<64>(p, grid, s);
 }
 
 rota_status rota_attn_get_error(void* stream) {
