@@ -192,7 +192,8 @@ def main():
     ap.add_argument("--workload", default="wan480")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-rows", type=int, default=128)
+    ap.add_argument("--ref-rows", type=int, default=128)      # per step of --impl reference
+    ap.add_argument("--cpu-rows", type=int, default=1024)     # the cpu_baseline sample (about 10 s)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -334,7 +335,7 @@ def main():
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = oracle_sample(w, q, k, v)
+            line["cpu_baseline"] = oracle_sample(w, q, k, v, rows=args.cpu_rows)
             line["cpu_baseline"].pop("seconds", None)
         print(json.dumps(line), flush=True)
     if pg is not None:
