@@ -193,7 +193,7 @@ const char* rota_attn_status_string(rota_status s);
  * every head takes the INT4 path (no FP16 fallback).  The intermediate codes,
  * scales and RoPE tables live in one 16 MiB array in the library's static
  * device memory, which every GPU that loads the library holds until exit.
- * Its size bounds the problem: B*H*nblk*(232*head_dim + 8) bytes of codes,
+ * Its size bounds the problem: B*H*nblk*(420*head_dim + 8) bytes of codes,
  * widened tiles and scales plus the RoPE tables (each entry padded to 256 bytes)
  * must fit in ROTA_NOALLOC_SCRATCH_BYTES, and each RoPE table in
  * ROTA_NOALLOC_MAX_TABLE floats; larger problems return
