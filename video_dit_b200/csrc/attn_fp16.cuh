@@ -11,7 +11,8 @@
 //   warp 0      TMA producer: the two Q tiles once, then the K and V tiles of
 //               each 64-key block (tensor-map loads straight from q_rope,
 //               k_rope and v, 128-byte swizzle) into a 3-stage ring;
-//   warp 1      TMEM owner and MMA issuer (one thread);
+//   warp 1      TMEM owner and MMA issuer (warp-uniform loop, one elected
+//               lane issues);
 //   warps 2-3   idle;
 //   warps 4-7   tile 0, warps 8-11 tile 1 (thread = row = TMEM lane).
 // S_t(j) = Q_t K_j^T (kind::f16, fp32 in TMEM, two buffers per tile).  O_t
@@ -131,45 +132,52 @@ __global__ void __launch_bounds__(kF16Threads, 1) attn_fp16_kernel(const __grid_
   const uint32_t tmem = *sTmem;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---- TMA producer ----
+    // ---- TMA producer (warp-uniform loop, one elected lane issues) ----
+    if (elect_one()) {
       mbar_arrive_expect_tx(q_full, 2 * L::Q_BYTES);
       for (int t = 0; t < 2; ++t)
         for (int a = 0; a < L::ATOMS; ++a)
           tma_load_2d(smem + L::OFF_Q + t * L::Q_BYTES + a * (kBM * 128), &p.tm_q, 64 * a, row_base + q0 + t * kBM,
                       q_full);
-      int issued = 0;
-      for (int j = 0; j < nkb; ++j) {
-        const int st = j % kF16Stages;
-        if (!mbar_wait(&kv_empty[st], ((j / kF16Stages) & 1) ^ 1, lim)) { *sAbort = 1; break; }
-        if (*sAbort) break;
-        uint8_t* kt = smem + L::OFF_KV + st * L::STAGE_BYTES;
+    }
+    __syncwarp();
+    int issued = 0;
+    for (int j = 0; j < nkb; ++j) {
+      const int st = j % kF16Stages;
+      if (!warp_wait(&kv_empty[st], ((j / kF16Stages) & 1) ^ 1, lim)) {
+        if (lane == 0) *sAbort = 1;
+        break;
+      }
+      if (warp_flag(sAbort)) break;
+      uint8_t* kt = smem + L::OFF_KV + st * L::STAGE_BYTES;
+      if (elect_one()) {
         mbar_arrive_expect_tx(&kv_full[st], L::STAGE_BYTES);
         for (int a = 0; a < L::ATOMS; ++a) {
           tma_load_2d(kt + a * (kBN * 128), &p.tm_k, 64 * a, row_base + j * kBN, &kv_full[st]);
           tma_load_2d(kt + L::K_BYTES + a * (kBN * 128), &p.tm_v, 64 * a, row_base + j * kBN, &kv_full[st]);
         }
-        issued = j + 1;
       }
-      // drain: every issued copy has landed before the CTA may exit
-      mbar_wait(q_full, 0, lim);
-      for (int j = (issued > kF16Stages ? issued - kF16Stages : 0); j < issued; ++j)
-        mbar_wait(&kv_full[j % kF16Stages], (j / kF16Stages) & 1, lim);
+      __syncwarp();
+      issued = j + 1;
     }
+    // drain: every issued copy has landed before the CTA may exit
+    warp_wait(q_full, 0, lim);
+    for (int j = (issued > kF16Stages ? issued - kF16Stages : 0); j < issued; ++j)
+      warp_wait(&kv_full[j % kF16Stages], (j / kF16Stages) & 1, lim);
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---- MMA issuer ----
-      constexpr uint32_t ID_S = idesc(1, 0, 0, kBM, kBN);     // f16 x f16 -> f32, 128 x 64
-      constexpr uint32_t ID_PV = idesc(1, 0, 0, kBM, D, 1);   // B (V) channels-contiguous
-      const uint32_t q_addr = smem_u32(smem + L::OFF_Q), kv_addr = smem_u32(smem + L::OFF_KV);
-      const uint32_t p_addr = smem_u32(smem + L::OFF_P);
-      bool ok = mbar_wait(q_full, 0, lim);
-      auto issue_s = [&](int j, int t) -> bool {
-        const int sb = 2 * t + (j & 1);
-        if (!mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1, lim)) return false;
-        tc_fence_after();
-        const uint32_t qa = q_addr + t * L::Q_BYTES, ka = kv_addr + (j % kF16Stages) * L::STAGE_BYTES;
-        const uint32_t d = tmem + L::T_S + sb * kBN;
+    // ---- MMA issuer (warp-uniform loop, one elected lane issues) ----
+    constexpr uint32_t ID_S = idesc(1, 0, 0, kBM, kBN);     // f16 x f16 -> f32, 128 x 64
+    constexpr uint32_t ID_PV = idesc(1, 0, 0, kBM, D, 1);   // B (V) channels-contiguous
+    const uint32_t q_addr = smem_u32(smem + L::OFF_Q), kv_addr = smem_u32(smem + L::OFF_KV);
+    const uint32_t p_addr = smem_u32(smem + L::OFF_P);
+    bool ok = warp_wait(q_full, 0, lim);
+    auto issue_s = [&](int j, int t) -> bool {
+      const int sb = 2 * t + (j & 1);
+      if (!warp_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1, lim)) return false;
+      tc_fence_after();
+      const uint32_t qa = q_addr + t * L::Q_BYTES, ka = kv_addr + (j % kF16Stages) * L::STAGE_BYTES;
+      const uint32_t d = tmem + L::T_S + sb * kBN;
+      if (elect_one()) {
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t atom = k >> 2, within = (k & 3) * 32;
@@ -177,39 +185,44 @@ __global__ void __launch_bounds__(kF16Threads, 1) attn_fp16_kernel(const __grid_
                   ID_S, k > 0);
         }
         mma_commit(&s_full[sb]);
-        return true;
-      };
-      auto issue_pv = [&](int j) -> bool {
-        const uint32_t va = kv_addr + (j % kF16Stages) * L::STAGE_BYTES + L::K_BYTES;
-        for (int t = 0; t < 2; ++t) {
-          const int pb = 2 * t + (j & 1);
-          if (!mbar_wait(&p_full[pb], (j >> 1) & 1, lim)) return false;
-          tc_fence_after();
-          const uint32_t pa = p_addr + pb * L::P_BYTES;
-          const uint32_t d = tmem + L::T_O + t * D;
+      }
+      __syncwarp();
+      return true;
+    };
+    auto issue_pv = [&](int j) -> bool {
+      const uint32_t va = kv_addr + (j % kF16Stages) * L::STAGE_BYTES + L::K_BYTES;
+      for (int t = 0; t < 2; ++t) {
+        const int pb = 2 * t + (j & 1);
+        if (!warp_wait(&p_full[pb], (j >> 1) & 1, lim)) return false;
+        tc_fence_after();
+        const uint32_t pa = p_addr + pb * L::P_BYTES;
+        const uint32_t d = tmem + L::T_O + t * D;
+        if (elect_one()) {
 #pragma unroll
           for (int k = 0; k < kBN / 16; ++k)
             mma_f16(d, sdesc(pa + 32 * k, 1024, 2), sdesc_lbo(va + 2048 * k, kBN * 128, 1024, 2), ID_PV,
                     (j > 0 || k > 0) ? 1u : 0u);
           mma_commit(&o_ready[t]);
           mma_commit(&p_empty[pb]);
+          if (t == 1) mma_commit(&kv_empty[j % kF16Stages]);
         }
-        mma_commit(&kv_empty[j % kF16Stages]);
-        return true;
-      };
-      for (int j = 0; ok && j < nkb; ++j) {
-        if (!mbar_wait(&kv_full[j % kF16Stages], (j / kF16Stages) & 1, lim)) { ok = false; break; }
-        tc_fence_after();
-        if (!issue_s(j, 0) || !issue_s(j, 1)) { ok = false; break; }
-        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
-        if (*sAbort) { ok = false; break; }
+        __syncwarp();
       }
-      if (ok) ok = issue_pv(nkb - 1);
-      if (!ok) *sAbort = 1;
-      // every issued MMA completes before TMEM is released
-      mma_commit(mma_done);
-      mbar_wait(mma_done, 0, lim);
+      return true;
+    };
+    for (int j = 0; ok && j < nkb; ++j) {
+      if (!warp_wait(&kv_full[j % kF16Stages], (j / kF16Stages) & 1, lim)) { ok = false; break; }
+      tc_fence_after();
+      if (!issue_s(j, 0) || !issue_s(j, 1)) { ok = false; break; }
+      if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+      if (warp_flag(sAbort)) { ok = false; break; }
     }
+    if (ok) ok = issue_pv(nkb - 1);
+    if (!ok && lane == 0) *sAbort = 1;
+    // every issued MMA completes before TMEM is released
+    if (elect_one()) mma_commit(mma_done);
+    __syncwarp();
+    warp_wait(mma_done, 0, lim);
   } else if (warp >= 4) {
     // ===================================================== query-tile warps
     const int t = (warp - 4) >> 2;       // tile 0 or 1

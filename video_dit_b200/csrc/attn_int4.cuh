@@ -34,7 +34,8 @@
 // One CTA = two 128-row query tiles of one head (256 rows), 384 threads:
 //   warp 0      TMA producer: the K, V'_hi and V'_lo tiles of each 64-key
 //               block -> a 3-stage shared-memory ring (cp.async.bulk);
-//   warp 1      TMEM owner and MMA issuer (one thread);
+//   warp 1      TMEM owner and MMA issuer (warp-uniform loop, one elected
+//               lane issues);
 //   warps 2-3   idle;
 //   warps 4-7   query tile 0, warps 8-11 query tile 1 (thread = row = TMEM lane):
 //               running max, P codes (fp16) and their row sum, O rescale,
@@ -220,25 +221,30 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     // ===================================================== producer warpgroup
     setmaxnreg_producer();
     if (warp == 0) {
-      if (lane == 0) {
-        // ---- TMA producer: widened tiles of block j -> operand stage j % kOps ----
-        int issued = 0;
-        for (int j = 0; j < nkb; ++j) {
-          const int op = j % kOps;
-          if (!mbar_wait(&op_empty[op], ((j / kOps) & 1) ^ 1, lim)) { *sAbort = 1; break; }
-          if (*sAbort) break;
-          uint8_t* dst = smem + L::OFF_OP + op * L::OP_BYTES;
-          const uint8_t* src = p.work + (head * p.nblk + j) * (size_t)L::IMG_BYTES;
+      // ---- TMA producer: widened tiles of block j -> operand stage j % kOps
+      // (warp-uniform loop, one elected lane issues the copies) ----
+      int issued = 0;
+      for (int j = 0; j < nkb; ++j) {
+        const int op = j % kOps;
+        if (!warp_wait(&op_empty[op], ((j / kOps) & 1) ^ 1, lim)) {
+          if (lane == 0) *sAbort = 1;
+          break;
+        }
+        if (warp_flag(sAbort)) break;
+        uint8_t* dst = smem + L::OFF_OP + op * L::OP_BYTES;
+        const uint8_t* src = p.work + (head * p.nblk + j) * (size_t)L::IMG_BYTES;
+        if (elect_one()) {
           mbar_arrive_expect_tx(&op_full[op], L::OP_BYTES);
           bulk_g2s(dst, src, L::K_BYTES, &op_full[op]);
           bulk_g2s(dst + L::K_BYTES, src + L::K_BYTES, L::VP_BYTES, &op_full[op]);
           bulk_g2s(dst + L::K_BYTES + L::VP_BYTES, src + L::K_BYTES + L::VP_BYTES, L::VP_BYTES, &op_full[op]);
-          issued = j + 1;
         }
-        // drain: every issued copy has landed before the CTA may exit
-        for (int j = (issued > kOps ? issued - kOps : 0); j < issued; ++j)
-          mbar_wait(&op_full[j % kOps], (j / kOps) & 1, lim);
+        __syncwarp();
+        issued = j + 1;
       }
+      // drain: every issued copy has landed before the CTA may exit
+      for (int j = (issued > kOps ? issued - kOps : 0); j < issued; ++j)
+        warp_wait(&op_full[j % kOps], (j / kOps) & 1, lim);
     } else if (warp == 1) {
       // ---- MMA issuer: the whole warp runs the loop, so addresses and waits
       // are warp-uniform; one elected lane issues each MMA and commit ----
