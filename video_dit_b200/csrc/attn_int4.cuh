@@ -34,9 +34,9 @@
 // One CTA = two 128-row query tiles of one head (256 rows), 384 threads:
 //   warp 0      TMA producer: the K, V'_hi and V'_lo tiles of each 64-key
 //               block -> a 3-stage shared-memory ring (cp.async.bulk);
-//   warp 1      TMEM owner and MMA issuer (warp-uniform loop, one elected
-//               lane issues);
-//   warps 2-3   idle;
+//   warps 1, 2  MMA issuers of tile 0 and tile 1 (warp-uniform loops, one
+//               elected lane issues); warp 1 also owns the TMEM allocation;
+//   warp 3      idle;
 //   warps 4-7   query tile 0, warps 8-11 query tile 1 (thread = row = TMEM lane):
 //               running max, P codes (fp16) and their row sum, O rescale,
 //               epilogue out = O / l.
@@ -101,8 +101,8 @@ struct Int4Smem {
   static constexpr int OFF_TAU = OFF_P + 4 * P_BYTES;
   static constexpr int OFF_BAR = OFF_TAU + 64;
   // barriers: op_full[3] op_empty[3] s_full[2 tiles] s_empty[2]
-  //           p_full[2 tiles][2 buffers] p_empty[2][2] q_full mma_done
-  static constexpr int NBAR = 3 + 3 + 2 + 2 + 4 + 4 + 1 + 1;
+  //           p_full[2 tiles][2 buffers] p_empty[2][2] q_full mma_done[2]
+  static constexpr int NBAR = 3 + 3 + 2 + 2 + 4 + 4 + 1 + 2;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int BYTES = OFF_ABORT + 4;
@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
   // holds every block up to that one (the MMAs of one thread run in order)
   uint64_t* p_empty = bars + 14;
   uint64_t* q_full = bars + 18;
-  uint64_t* mma_done = bars + 19;
+  uint64_t* mma_done = bars + 19;   // [2], one per MMA warp
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + L::OFF_ABORT);
   float* sTau = reinterpret_cast<float*>(smem + L::OFF_TAU);
@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
   if (tid == 0) {
     for (int i = 0; i < kOps; ++i) {
       mbar_init(&op_full[i], 1);
-      mbar_init(&op_empty[i], 1);
+      mbar_init(&op_empty[i], 2);   // the last P V of the block, one commit per tile
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&p_full[i], 4);
@@ -203,7 +203,8 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       mbar_init(&s_empty[t], 4);
     }
     mbar_init(q_full, 8);
-    mbar_init(mma_done, 1);
+    mbar_init(&mma_done[0], 1);
+    mbar_init(&mma_done[1], 1);
     *sAbort = 0;
     fence_mbar_init();
   }
@@ -245,72 +246,71 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       // drain: every issued copy has landed before the CTA may exit
       for (int j = (issued > kOps ? issued - kOps : 0); j < issued; ++j)
         warp_wait(&op_full[j % kOps], (j / kOps) & 1, lim);
-    } else if (warp == 1) {
-      // ---- MMA issuer: the whole warp runs the loop, so addresses and waits
-      // are warp-uniform; one elected lane issues each MMA and commit ----
+    } else if (warp <= 2) {
+      // ---- MMA issuers: warp 1 + t issues tile t's MMAs, so the two tiles'
+      // S -> softmax -> P V chains do not wait on each other.  The whole warp
+      // runs the loop (addresses and waits warp-uniform); one elected lane
+      // issues each MMA and commit ----
+      const int t = warp - 1;
       constexpr uint32_t ID_S = idesc(1, 0, 0, kBM, kBN);   // e4m3 x e4m3 -> f32, 128 x 64
       constexpr uint32_t ID_PV = idesc(1, 0, 0, kBM, D);    // f16 x f16 -> f32, 128 x D
       // descriptors: constant high words, low words stepped by 32 bytes (2 units) per K step
       const uint32_t hi_qk = sdesc_hi(L::SBO_QK, L::LAYOUT_QK), hi_128 = sdesc_hi(1024, 2);
       const uint32_t lo_p = sdesc_lo(smem_u32(smem + L::OFF_P));    // + (2t + (j & 1)) * P_BYTES / 16
       const uint32_t lo_op = sdesc_lo(smem_u32(smem + L::OFF_OP));  // + op * OP_BYTES / 16
+      const uint32_t aq = tmem + L::T_Q + t * (D / 4);   // Q of tile t: 32 e4m3 elements = 8 columns per K step
+      const uint32_t d_s = tmem + L::T_S + t * kBN, d_o = tmem + L::T_O + t * D;
       bool ok = warp_wait(q_full, 0, lim);
-      auto issue_s = [&](int j, int t) -> bool {
+      auto issue_s = [&](int j) -> bool {
         const int op = j % kOps;
         if (!warp_wait(&s_empty[t], (j & 1) ^ 1, lim)) return false;
         tc_fence_after();
         if (p.inject_skip && j == 0 && t == 0) return true;  // fault injection: never committed
         const uint32_t lk = lo_op + op * (L::OP_BYTES >> 4);
-        const uint32_t aq = tmem + L::T_Q + t * (D / 4);   // 32 e4m3 elements = 8 columns per K step
-        const uint32_t d = tmem + L::T_S + t * kBN;
         if (elect_one()) {
-          mma_f8f6f4_ts<0>(d, aq, lk, hi_qk, ID_S);
+          mma_f8f6f4_ts<0>(d_s, aq, lk, hi_qk, ID_S);
 #pragma unroll
-          for (int k = 1; k < D / 32; ++k) mma_f8f6f4_ts<1>(d, aq + 8 * k, lk + 2 * k, hi_qk, ID_S);
+          for (int k = 1; k < D / 32; ++k) mma_f8f6f4_ts<1>(d_s, aq + 8 * k, lk + 2 * k, hi_qk, ID_S);
           mma_commit(&s_full[t]);
         }
         __syncwarp();
         return true;
       };
       auto issue_pv = [&](int j) -> bool {
-        const int op = j % kOps;
+        const int op = j % kOps, pb = 2 * t + (j & 1);
         const uint32_t lvh = lo_op + op * (L::OP_BYTES >> 4) + (L::K_BYTES >> 4);
         const uint32_t lvl = lvh + (L::VP_BYTES >> 4);
-        for (int t = 0; t < 2; ++t) {
-          const int pb = 2 * t + (j & 1);
-          if (!warp_wait(&p_full[pb], (j >> 1) & 1, lim)) return false;
-          tc_fence_after();
-          const uint32_t lp = lo_p + pb * (L::P_BYTES >> 4);
-          const uint32_t d = tmem + L::T_O + t * D;
-          if (elect_one()) {
-            if (j == 0) mma_f16_lh<0>(d, lp, hi_128, lvh, hi_128, ID_PV);
-            else mma_f16_lh<1>(d, lp, hi_128, lvh, hi_128, ID_PV);
-            mma_f16_lh<1>(d, lp, hi_128, lvl, hi_128, ID_PV);
+        if (!warp_wait(&p_full[pb], (j >> 1) & 1, lim)) return false;
+        tc_fence_after();
+        const uint32_t lp = lo_p + pb * (L::P_BYTES >> 4);
+        if (elect_one()) {
+          if (j == 0) mma_f16_lh<0>(d_o, lp, hi_128, lvh, hi_128, ID_PV);
+          else mma_f16_lh<1>(d_o, lp, hi_128, lvh, hi_128, ID_PV);
+          mma_f16_lh<1>(d_o, lp, hi_128, lvl, hi_128, ID_PV);
 #pragma unroll
-            for (int k = 1; k < kBN / 16; ++k) {
-              mma_f16_lh<1>(d, lp + 2 * k, hi_128, lvh + 2 * k, hi_128, ID_PV);
-              mma_f16_lh<1>(d, lp + 2 * k, hi_128, lvl + 2 * k, hi_128, ID_PV);
-            }
-            mma_commit(&p_empty[pb]);
-            if (t == 1) mma_commit(&op_empty[op]);
+          for (int k = 1; k < kBN / 16; ++k) {
+            mma_f16_lh<1>(d_o, lp + 2 * k, hi_128, lvh + 2 * k, hi_128, ID_PV);
+            mma_f16_lh<1>(d_o, lp + 2 * k, hi_128, lvl + 2 * k, hi_128, ID_PV);
           }
-          __syncwarp();
+          mma_commit(&p_empty[pb]);
+          mma_commit(&op_empty[op]);   // one of the stage's two arrivals (one per tile)
         }
+        __syncwarp();
         return true;
       };
       for (int j = 0; ok && j < nkb; ++j) {
         if (!warp_wait(&op_full[j % kOps], (j / kOps) & 1, lim)) { ok = false; break; }
         tc_fence_after();
-        if (!issue_s(j, 0) || !issue_s(j, 1)) { ok = false; break; }
+        if (!issue_s(j)) { ok = false; break; }
         if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
         if (warp_flag(sAbort)) { ok = false; break; }
       }
       if (ok) ok = issue_pv(nkb - 1);
       if (!ok && lane == 0) *sAbort = 1;
-      // every issued MMA completes before TMEM is released
-      if (elect_one()) mma_commit(mma_done);
+      // every MMA this warp issued completes before TMEM is released
+      if (elect_one()) mma_commit(&mma_done[t]);
       __syncwarp();
-      warp_wait(mma_done, 0, lim);
+      warp_wait(&mma_done[t], 0, lim);
     }
   } else {
     // ===================================================== query-tile warpgroups
