@@ -95,26 +95,25 @@ struct Int4Smem {
   static constexpr int VP_BYTES = D * kBN * 2;                    // one V' part: D rows x 64 keys fp16
   static constexpr int OP_BYTES = K_BYTES + 2 * VP_BYTES;
   static constexpr int IMG_BYTES = OP_BYTES;                      // one block in int4_work
-  static constexpr int P_BYTES = kBM * kBN * 2;                   // P codes, fp16 [128 rows x 128 B]
   static constexpr int OFF_OP = 0;                                // kOps stages
-  static constexpr int OFF_P = OFF_OP + kOps * OP_BYTES;          // 2 tiles x 2 buffers
-  static constexpr int OFF_TAU = OFF_P + 4 * P_BYTES;
+  static constexpr int OFF_TAU = OFF_OP + kOps * OP_BYTES;
   static constexpr int OFF_BAR = OFF_TAU + 64;
-  // barriers: op_full[3] op_empty[3] s_full[2 tiles] s_empty[2]
-  //           p_full[2 tiles][2 buffers] p_empty[2][2] q_full mma_done[2]
-  static constexpr int NBAR = 3 + 3 + 2 + 2 + 4 + 4 + 1 + 2;
+  // barriers: op_full[3] op_empty[3] s_full[2 tiles] s_empty[2] p_full[2]
+  //           p_empty[2] q_full mma_done[2]
+  static constexpr int NBAR = 3 + 3 + 2 + 2 + 2 + 2 + 1 + 2;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int BYTES = OFF_ABORT + 4;
   static constexpr int ALLOC = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   // S of tile t at column t * 64; the e4m3 Q rows of tile t (A operand of the
-  // score MMA) at 128 + t * D / 4; O of tile t at 256 + t * D
-  static constexpr uint32_t T_S = 0, T_Q = 2 * kBN, T_O = 4 * kBN;
-  static_assert(T_Q + 2 * (D / 4) <= T_O && T_O + 2 * D <= TMEM_COLS, "TMEM budget");
+  // score MMA) at 128 + t * D / 4; the fp16 P codes of tile t (A operand of
+  // P V, 64 keys = 32 columns) at 192 + 32 t; O of tile t at 256 + t * D
+  static constexpr uint32_t T_S = 0, T_Q = 2 * kBN, T_P = 192, T_O = 4 * kBN;
+  static_assert(T_Q + 2 * (D / 4) <= T_P && T_P + 2 * (kBN / 2) <= T_O && T_O + 2 * D <= TMEM_COLS,
+                "TMEM budget");
   static_assert(IMG_BYTES % 16 == 0 && K_BYTES % 16 == 0 && VP_BYTES % 16 == 0, "bulk copy sizes");
-  static_assert(OFF_OP % 1024 == 0 && OP_BYTES % 1024 == 0 && K_BYTES % 1024 == 0 && VP_BYTES % 1024 == 0 &&
-                    OFF_P % 1024 == 0 && P_BYTES % 1024 == 0,
+  static_assert(OFF_OP % 1024 == 0 && OP_BYTES % 1024 == 0 && K_BYTES % 1024 == 0 && VP_BYTES % 1024 == 0,
                 "swizzle atom alignment");
   static_assert(ALLOC <= 232448, "shared memory budget");
 };
@@ -166,16 +165,15 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* op_full = bars;
   uint64_t* op_empty = bars + 3;
-  uint64_t* s_full = bars + 6;     // per tile, once per block
+  // per tile, once per block (phase j & 1)
+  uint64_t* s_full = bars + 6;
   uint64_t* s_empty = bars + 8;
-  // per (tile t, buffer b) = index 2t + b, buffer b = block parity: each
-  // completes once per use of its buffer (phase (j >> 1) & 1 for block j)
   uint64_t* p_full = bars + 10;
-  // p_empty[2t + b]: the P V that read P buffer 2t + b has completed -- so O
-  // holds every block up to that one (the MMAs of one thread run in order)
-  uint64_t* p_empty = bars + 14;
-  uint64_t* q_full = bars + 18;
-  uint64_t* mma_done = bars + 19;   // [2], one per MMA warp
+  // p_empty[t]: tile t's P V of the block has completed -- the P columns may
+  // be rewritten, and O holds every block up to that one
+  uint64_t* p_empty = bars + 12;
+  uint64_t* q_full = bars + 14;
+  uint64_t* mma_done = bars + 15;   // [2], one per MMA warp
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + L::OFF_ABORT);
   float* sTau = reinterpret_cast<float*>(smem + L::OFF_TAU);
@@ -194,13 +192,11 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       mbar_init(&op_full[i], 1);
       mbar_init(&op_empty[i], 2);   // the last P V of the block, one commit per tile
     }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&p_full[i], 4);
-      mbar_init(&p_empty[i], 1);
-    }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&s_empty[t], 4);
+      mbar_init(&p_full[t], 4);
+      mbar_init(&p_empty[t], 1);
     }
     mbar_init(q_full, 8);
     mbar_init(&mma_done[0], 1);
@@ -256,7 +252,6 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       constexpr uint32_t ID_PV = idesc(1, 0, 0, kBM, D);    // f16 x f16 -> f32, 128 x D
       // descriptors: constant high words, low words stepped by 32 bytes (2 units) per K step
       const uint32_t hi_qk = sdesc_hi(L::SBO_QK, L::LAYOUT_QK), hi_128 = sdesc_hi(1024, 2);
-      const uint32_t lo_p = sdesc_lo(smem_u32(smem + L::OFF_P));    // + (2t + (j & 1)) * P_BYTES / 16
       const uint32_t lo_op = sdesc_lo(smem_u32(smem + L::OFF_OP));  // + op * OP_BYTES / 16
       const uint32_t aq = tmem + L::T_Q + t * (D / 4);   // Q of tile t: 32 e4m3 elements = 8 columns per K step
       const uint32_t d_s = tmem + L::T_S + t * kBN, d_o = tmem + L::T_O + t * D;
@@ -276,23 +271,23 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         __syncwarp();
         return true;
       };
+      const uint32_t ap = tmem + L::T_P + t * (kBN / 2);   // P of tile t: 16 keys = 8 columns per K step
       auto issue_pv = [&](int j) -> bool {
-        const int op = j % kOps, pb = 2 * t + (j & 1);
+        const int op = j % kOps;
         const uint32_t lvh = lo_op + op * (L::OP_BYTES >> 4) + (L::K_BYTES >> 4);
         const uint32_t lvl = lvh + (L::VP_BYTES >> 4);
-        if (!warp_wait(&p_full[pb], (j >> 1) & 1, lim)) return false;
+        if (!warp_wait(&p_full[t], j & 1, lim)) return false;
         tc_fence_after();
-        const uint32_t lp = lo_p + pb * (L::P_BYTES >> 4);
         if (elect_one()) {
-          if (j == 0) mma_f16_lh<0>(d_o, lp, hi_128, lvh, hi_128, ID_PV);
-          else mma_f16_lh<1>(d_o, lp, hi_128, lvh, hi_128, ID_PV);
-          mma_f16_lh<1>(d_o, lp, hi_128, lvl, hi_128, ID_PV);
+          if (j == 0) mma_f16_ts<0>(d_o, ap, lvh, hi_128, ID_PV);
+          else mma_f16_ts<1>(d_o, ap, lvh, hi_128, ID_PV);
+          mma_f16_ts<1>(d_o, ap, lvl, hi_128, ID_PV);
 #pragma unroll
           for (int k = 1; k < kBN / 16; ++k) {
-            mma_f16_lh<1>(d_o, lp + 2 * k, hi_128, lvh + 2 * k, hi_128, ID_PV);
-            mma_f16_lh<1>(d_o, lp + 2 * k, hi_128, lvl + 2 * k, hi_128, ID_PV);
+            mma_f16_ts<1>(d_o, ap + 8 * k, lvh + 2 * k, hi_128, ID_PV);
+            mma_f16_ts<1>(d_o, ap + 8 * k, lvl + 2 * k, hi_128, ID_PV);
           }
-          mma_commit(&p_empty[pb]);
+          mma_commit(&p_empty[t]);
           mma_commit(&op_empty[op]);   // one of the stage's two arrivals (one per tile)
         }
         __syncwarp();
@@ -321,6 +316,7 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     const uint32_t t_lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + L::T_S + t * kBN + t_lane;
     const uint32_t tO = tmem + L::T_O + t * D + t_lane;
+    const uint32_t tP = tmem + L::T_P + t * (kBN / 2) + t_lane;
 
     // own Q row: packed codes -> e4m3 subnormals, K-contiguous in this lane's
     // TMEM columns (the A operand of the score MMA)
@@ -351,7 +347,6 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     for (int j = 0; j < nkb; ++j) {
       const float sk = sk_next;
       if (j + 1 < nkb) sk_next = __ldg(ksc + j + 1);
-      const int sb = 2 * t + (j & 1);   // P buffer
       if (!warp_wait(&s_full[t], j & 1, lim)) { aborted = true; break; }
       tc_fence_after();
 
@@ -416,53 +411,20 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         near = fmaxf(n0, n1);
         lsum = ls0 + ls1;
       }
-      // the P V that read this buffer (block j - 2) has completed
-      if (j >= 2 && !warp_wait(&p_empty[sb], ((j >> 1) & 1) ^ 1, lim)) { aborted = true; break; }
-      uint8_t* sP = smem + L::OFF_P + sb * L::P_BYTES;
-#pragma unroll
-      for (int k = 0; k < kBN / 8; ++k)
-        *reinterpret_cast<uint4*>(sP + swz<128>(r, 16 * k)) =
-            make_uint4(pw[2 * k].x, pw[2 * k].y, pw[2 * k + 1].x, pw[2 * k + 1].y);
-
-      // ---- exact decisions (rare): estimates within 1e-5 of a half-integer ----
-      // Recompute which keys were near a tie (same arithmetic as above), then
-      // visit only the columns some lane flagged; S is still in TMEM.
-      if (__any_sync(0xffffffffu, near > kNear)) {
-        uint32_t mlo = 0, mhi = 0;
-#pragma unroll
-        for (int k = 0; k < kBN; ++k) {
-          const float d = __fmaf_rn(__uint_as_float(sr[k]), c18, -m);
-          const float e = ex2_approx(d);
-          const float rr = __fadd_rn(__fmaf_rn(e, 15.f, kMagic), -kMagic);
-          const bool hit = fabsf(__fmaf_rn(e, 15.f, -rr)) > kNear;
-          if (k < 32) mlo |= static_cast<uint32_t>(hit) << k;
-          else mhi |= static_cast<uint32_t>(hit) << (k - 32);
-        }
-        uint32_t wlo = __reduce_or_sync(0xffffffffu, mlo), whi = __reduce_or_sync(0xffffffffu, mhi);
-        while (wlo | whi) {
-          const int k = wlo ? __ffs(wlo) - 1 : 32 + __ffs(whi) - 1;
-          if (k < 32) wlo &= wlo - 1; else whi &= whi - 1;
-          uint32_t sbits = 0;
-#pragma unroll
-          for (int kk = 0; kk < kBN; ++kk) sbits = kk == k ? sr[kk] : sbits;
-          const bool mine = (k < 32 ? (mlo >> k) : (mhi >> (k - 32))) & 1u;
-          if (mine) {
-            const float d = __fmaf_rn(__uint_as_float(sbits), c18, -m);
-            const float e = ex2_approx(d);
-            const float rr = __fadd_rn(__fmaf_rn(e, 15.f, kMagic), -kMagic);
-            const float u = pcode_f(d, sTau);
-            lsum += u - rr;
-            *reinterpret_cast<__half*>(sP + swz<128>(r, 2 * k)) = __float2half_rn(u);
-          }
-        }
-      }
       // keys past N in the last block take code 0; the row sum is taken again
       if (nvalid < kBN) {
         lsum = 0.f;
-        for (int k = 0; k < kBN; ++k) {
-          __half* hk = reinterpret_cast<__half*>(sP + swz<128>(r, 2 * k));
-          if (k >= nvalid) *hk = __float2half_rn(0.f);
-          lsum += __half2float(*hk);
+#pragma unroll
+        for (int w = 0; w < kBN / 4; ++w) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int sh = 16 * (e & 1);
+            uint32_t word = (e & 2) ? pw[w].y : pw[w].x;
+            if (4 * w + e >= nvalid) word &= ~(0xFFFFu << sh);
+            lsum += __half2float(__ushort_as_half(static_cast<unsigned short>((word >> sh) & 0xFFFFu)));
+            if (e & 2) pw[w].y = word;
+            else pw[w].x = word;
+          }
         }
       }
       if (DUMP) {
@@ -473,12 +435,14 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
                 static_cast<int32_t>(__uint_as_float(sr[k]) * 262144.f);
       }
 
-      // ---- the running max moved on some row of the warp: rescale O and l ----
-      l = __fmaf_rn(l, alpha, lsum);
-      if (j > 0 && !__all_sync(0xffffffffu, alpha == 1.f)) {
-        // the previous block's P V has landed in O
-        if (!warp_wait(&p_empty[2 * t + ((j - 1) & 1)], ((j - 1) >> 1) & 1, lim)) { aborted = true; break; }
+      // the previous block's P V has completed: its P columns are free and O
+      // holds every block before this one
+      if (j > 0) {
+        if (!warp_wait(&p_empty[t], (j - 1) & 1, lim)) { aborted = true; break; }
         tc_fence_after();
+      }
+      // ---- the running max moved on some row of the warp: rescale O ----
+      if (j > 0 && !__all_sync(0xffffffffu, alpha == 1.f)) {
 #pragma unroll 1
         for (int cb = 0; cb < D / 32; ++cb) {
           uint32_t o[32];
@@ -488,23 +452,78 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
           for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__fmul_rn(__uint_as_float(o[k]), alpha));
           tmem_st32(tO + 32 * cb, o);
         }
-        tmem_st_wait();
       }
-      fence_proxy_async_smem();
+      // P codes -> this lane's TMEM columns (keys 2c, 2c + 1 in column c)
+      {
+        uint32_t pr[kBN / 2];
+#pragma unroll
+        for (int w = 0; w < kBN / 4; ++w) {
+          pr[2 * w] = pw[w].x;
+          pr[2 * w + 1] = pw[w].y;
+        }
+        tmem_st32(tP, pr);
+      }
+      // ---- exact decisions (rare): estimates within 1e-5 of a half-integer ----
+      // Recompute which keys were near a tie (same arithmetic as above), then
+      // visit only the columns some lane flagged: each is read back from TMEM,
+      // the flagged lanes put in the exact code, and it is stored again.
+      if (__any_sync(0xffffffffu, near > kNear)) {
+        tmem_st_wait();
+        uint32_t mlo = 0, mhi = 0;
+#pragma unroll
+        for (int k = 0; k < kBN; ++k) {
+          const float d = __fmaf_rn(__uint_as_float(sr[k]), c18, -m);
+          const float e = ex2_approx(d);
+          const float rr = __fadd_rn(__fmaf_rn(e, 15.f, kMagic), -kMagic);
+          const bool hit = fabsf(__fmaf_rn(e, 15.f, -rr)) > kNear && k < nvalid;
+          if (k < 32) mlo |= static_cast<uint32_t>(hit) << k;
+          else mhi |= static_cast<uint32_t>(hit) << (k - 32);
+        }
+        uint32_t wlo = __reduce_or_sync(0xffffffffu, mlo), whi = __reduce_or_sync(0xffffffffu, mhi);
+        while (wlo | whi) {
+          const int k = wlo ? __ffs(wlo) - 1 : 32 + __ffs(whi) - 1;
+          if (k < 32) wlo &= wlo - 1; else whi &= whi - 1;
+          uint32_t sbits = 0;
+#pragma unroll
+          for (int kk = 0; kk < kBN; ++kk) sbits = kk == k ? sr[kk] : sbits;
+          uint32_t word = tmem_ld1(tP + (k >> 1));
+          tmem_wait_dep1(word);
+          const bool mine = (k < 32 ? (mlo >> k) : (mhi >> (k - 32))) & 1u;
+          if (mine) {
+            const float d = __fmaf_rn(__uint_as_float(sbits), c18, -m);
+            const float e = ex2_approx(d);
+            const float rr = __fadd_rn(__fmaf_rn(e, 15.f, kMagic), -kMagic);
+            const float u = pcode_f(d, sTau);
+            lsum += u - rr;
+            const int sh = 16 * (k & 1);
+            word = (word & ~(0xFFFFu << sh)) | (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(u))) << sh);
+          }
+          tmem_st1(tP + (k >> 1), word);
+          tmem_st_wait();
+        }
+      }
+      l = __fmaf_rn(l, alpha, lsum);
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
-      if (DUMP && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr) {
-        // P codes as the MMA will read them, from the fp16 values
+      if (lane == 0) mbar_arrive(&p_full[t]);
+      if (DUMP) {
+        // P codes as the MMA will read them, from the fp16 values in TMEM
         const size_t base = (size_t)(row - p.dbg_r0) * p.N + (size_t)j * kBN;
-        for (int k = 0; k < nvalid; ++k)
-          p.p_dump[base + k] =
-              static_cast<uint8_t>(__half2float(*reinterpret_cast<const __half*>(sP + swz<128>(r, 2 * k))));
+        for (int c2 = 0; c2 < kBN / 2; ++c2) {
+          uint32_t word = tmem_ld1(tP + c2);
+          tmem_wait_dep1(word);
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            if (2 * c2 + e < nvalid && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr)
+              p.p_dump[base + 2 * c2 + e] = static_cast<uint8_t>(
+                  __half2float(__ushort_as_half(static_cast<unsigned short>((word >> (16 * e)) & 0xFFFFu))));
+        }
       }
       if (warp_flag(sAbort)) { aborted = true; break; }
     }
     // ---- epilogue: out = O / l once the last P V has landed ----
-    if (!aborted && !warp_wait(&p_empty[2 * t + ((nkb - 1) & 1)], ((nkb - 1) >> 1) & 1, lim)) aborted = true;
+    if (!aborted && !warp_wait(&p_empty[t], (nkb - 1) & 1, lim)) aborted = true;
     if (aborted) {
       *sAbort = 1;
     } else {

@@ -266,6 +266,19 @@ __device__ __forceinline__ void mma_f16_lh(uint32_t d_tmem, uint32_t alo, uint32
       : "memory");
 }
 
+// kind::f16 with the A operand in TMEM (lane = row, two 16-bit elements per
+// 32-bit column, K-contiguous) and B by descriptor halves.
+template <int ACC>
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t blo, uint32_t bhi, uint32_t id) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 b;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "mov.b64 b, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(blo), "r"(bhi), "n"(ACC), "r"(id)
+      : "memory");
+}
+
 // Low word of a shared-memory descriptor: start address >> 4 and the (unused)
 // leading byte offset; the high word depends only on the layout.
 __device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr) { return ((saddr & 0x3FFFFu) >> 4) | (1u << 16); }
@@ -334,6 +347,10 @@ __device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t (&r)[N]
   static_assert(N == 16 || N == 32, "tcgen05.st shape");
   if constexpr (N == 32) tmem_st32(taddr, r);
   else tmem_st16(taddr, r);
+}
+// One 32-bit column per lane, register -> TMEM (dynamic column address allowed).
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
