@@ -10,14 +10,16 @@
 // One CTA = two 128-row query tiles of one flagged head, 384 threads:
 //   warp 0      TMA producer: the two Q tiles once, then the K and V tiles of
 //               each 64-key block (tensor-map loads straight from q_rope,
-//               k_rope and v, 128-byte swizzle) into a 3-stage ring;
-//   warp 1      TMEM owner and MMA issuer (warp-uniform loop, one elected
-//               lane issues);
-//   warps 2-3   idle;
+//               k_rope and v, 128-byte swizzle) into a 4-stage ring;
+//   warps 1, 2  MMA issuers of tile 0 and tile 1 (warp-uniform loops, one
+//               elected lane issues); warp 1 also owns the TMEM allocation;
+//   warp 3      idle;
 //   warps 4-7   tile 0, warps 8-11 tile 1 (thread = row = TMEM lane).
-// S_t(j) = Q_t K_j^T (kind::f16, fp32 in TMEM, two buffers per tile).  O_t
-// accumulates in TMEM across blocks: the MMA adds P_t(j) V_j to it, where V_j
-// is read as it sits in memory (channels contiguous: an MN-major B operand).
+// S_t(j) = Q_t K_j^T (kind::f16, fp32 in TMEM; the softmax warps release it
+// as soon as it is in registers).  P_t(j) goes to TMEM (tcgen05.st) and O_t
+// accumulates in TMEM across blocks: the MMA adds P_t(j) V_j to it, with P
+// read from TMEM and V_j as it sits in memory (channels contiguous: an
+// MN-major B operand).
 // The exponentials use a reference max m_ref per row that is raised only when
 // a block's max exceeds it by more than 8 (log2 units): P stays <= 2^8, which
 // fp16 holds, and O and l are rescaled in place only then (a warp rescales
@@ -44,7 +46,7 @@ struct Fp16Params {
 };
 
 constexpr int kF16Threads = 384;
-constexpr int kF16Stages = 3;
+constexpr int kF16Stages = 4;
 constexpr float kRescaleLog2 = 8.f;   // raise the reference max only past this margin
 
 template <int D>
@@ -54,24 +56,23 @@ struct F16Smem {
   static constexpr int K_BYTES = kBN * D * 2;          // ATOMS x [64 keys x 128 B], K-major
   static constexpr int V_BYTES = kBN * D * 2;          // ATOMS x [64 keys x 128 B], channels contiguous
   static constexpr int STAGE_BYTES = K_BYTES + V_BYTES;
-  static constexpr int P_BYTES = kBM * kBN * 2;        // [128 rows x 128 B]
   static constexpr int OFF_Q = 0;                                // 2 tiles
   static constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;             // kF16Stages stages
-  static constexpr int OFF_P = OFF_KV + kF16Stages * STAGE_BYTES;  // 2 tiles x 2 buffers
-  static constexpr int OFF_BAR = OFF_P + 4 * P_BYTES;
-  // barriers: kv_full[3] kv_empty[3] s_full[4] s_empty[4] p_full[4] p_empty[4]
-  //           o_ready[2] q_full mma_done
-  static constexpr int NBAR = 3 + 3 + 4 + 4 + 4 + 4 + 2 + 1 + 1;
+  static constexpr int OFF_BAR = OFF_KV + kF16Stages * STAGE_BYTES;
+  // barriers: kv_full[4] kv_empty[4] s_full[2 tiles] s_empty[2] p_full[2]
+  //           p_empty[2] q_full mma_done[2]
+  static constexpr int NBAR = 4 + 4 + 2 + 2 + 2 + 2 + 1 + 2;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int BYTES = OFF_ABORT + 4;
   static constexpr int ALLOC = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  // S of tile t, buffer b at column (2t + b) * 64; O of tile t at 256 + t * D
-  static constexpr uint32_t T_S = 0, T_O = 4 * kBN;
-  static_assert(T_O + 2 * D <= TMEM_COLS, "TMEM budget");
+  // S of tile t at column t * 64; the fp16 P of tile t (A operand of P V,
+  // 64 keys = 32 columns) at 128 + 32 t; O of tile t at 256 + t * D
+  static constexpr uint32_t T_S = 0, T_P = 2 * kBN, T_O = 4 * kBN;
+  static_assert(T_P + 2 * (kBN / 2) <= T_O && T_O + 2 * D <= TMEM_COLS, "TMEM budget");
   static_assert(ALLOC <= 232448, "shared memory budget");
-  static_assert(Q_BYTES % 1024 == 0 && K_BYTES % 1024 == 0 && P_BYTES % 1024 == 0, "swizzle atom alignment");
+  static_assert(Q_BYTES % 1024 == 0 && K_BYTES % 1024 == 0, "swizzle atom alignment");
 };
 
 template <int D>
@@ -81,16 +82,16 @@ __global__ void __launch_bounds__(kF16Threads, 1) attn_fp16_kernel(const __grid_
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* kv_full = bars;
-  uint64_t* kv_empty = bars + 3;
-  // per (tile t, buffer b) = index 2t + b, buffer b = block parity: each
-  // completes once per use of its buffer (phase (j >> 1) & 1 for block j)
-  uint64_t* s_full = bars + 6;
+  uint64_t* kv_empty = bars + 4;
+  // per tile, once per block (phase j & 1)
+  uint64_t* s_full = bars + 8;
   uint64_t* s_empty = bars + 10;
-  uint64_t* p_full = bars + 14;
-  uint64_t* p_empty = bars + 18;   // the P V that read P buffer 2t + b has completed
-  uint64_t* o_ready = bars + 22;   // P_t(j) V_j has completed (once per block)
-  uint64_t* q_full = bars + 24;
-  uint64_t* mma_done = bars + 25;
+  uint64_t* p_full = bars + 12;
+  // p_empty[t]: tile t's P V of the block has completed -- the P columns may
+  // be rewritten, and O holds every block up to that one
+  uint64_t* p_empty = bars + 14;
+  uint64_t* q_full = bars + 16;
+  uint64_t* mma_done = bars + 17;   // [2], one per MMA warp
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + L::OFF_ABORT);
 
@@ -106,18 +107,16 @@ __global__ void __launch_bounds__(kF16Threads, 1) attn_fp16_kernel(const __grid_
   if (tid == 0) {
     for (int i = 0; i < kF16Stages; ++i) {
       mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&kv_empty[i], 2);   // the last P V of the block, one commit per tile
     }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
-      mbar_init(&p_full[i], 4);
-      mbar_init(&p_empty[i], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&s_empty[t], 4);
+      mbar_init(&p_full[t], 4);
+      mbar_init(&p_empty[t], 1);
+      mbar_init(&mma_done[t], 1);
     }
-    mbar_init(&o_ready[0], 1);
-    mbar_init(&o_ready[1], 1);
     mbar_init(q_full, 1);
-    mbar_init(mma_done, 1);
     *sAbort = 0;
     fence_mbar_init();
   }
@@ -164,82 +163,79 @@ __global__ void __launch_bounds__(kF16Threads, 1) attn_fp16_kernel(const __grid_
     warp_wait(q_full, 0, lim);
     for (int j = (issued > kF16Stages ? issued - kF16Stages : 0); j < issued; ++j)
       warp_wait(&kv_full[j % kF16Stages], (j / kF16Stages) & 1, lim);
-  } else if (warp == 1) {
-    // ---- MMA issuer (warp-uniform loop, one elected lane issues) ----
+  } else if (warp <= 2) {
+    // ---- MMA issuers: warp 1 + t issues tile t's MMAs (warp-uniform loop,
+    // one elected lane issues) ----
+    const int t = warp - 1;
     constexpr uint32_t ID_S = idesc(1, 0, 0, kBM, kBN);     // f16 x f16 -> f32, 128 x 64
     constexpr uint32_t ID_PV = idesc(1, 0, 0, kBM, D, 1);   // B (V) channels-contiguous
-    const uint32_t q_addr = smem_u32(smem + L::OFF_Q), kv_addr = smem_u32(smem + L::OFF_KV);
-    const uint32_t p_addr = smem_u32(smem + L::OFF_P);
+    const uint32_t qa = smem_u32(smem + L::OFF_Q) + t * L::Q_BYTES, kv_addr = smem_u32(smem + L::OFF_KV);
+    const uint32_t d_s = tmem + L::T_S + t * kBN, d_o = tmem + L::T_O + t * D;
+    const uint32_t ap = tmem + L::T_P + t * (kBN / 2);   // P of tile t: 16 keys = 8 columns per K step
     bool ok = warp_wait(q_full, 0, lim);
-    auto issue_s = [&](int j, int t) -> bool {
-      const int sb = 2 * t + (j & 1);
-      if (!warp_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1, lim)) return false;
+    auto issue_s = [&](int j) -> bool {
+      if (!warp_wait(&s_empty[t], (j & 1) ^ 1, lim)) return false;
       tc_fence_after();
-      const uint32_t qa = q_addr + t * L::Q_BYTES, ka = kv_addr + (j % kF16Stages) * L::STAGE_BYTES;
-      const uint32_t d = tmem + L::T_S + sb * kBN;
+      const uint32_t ka = kv_addr + (j % kF16Stages) * L::STAGE_BYTES;
       if (elect_one()) {
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t atom = k >> 2, within = (k & 3) * 32;
-          mma_f16(d, sdesc(qa + atom * (kBM * 128) + within, 1024, 2), sdesc(ka + atom * (kBN * 128) + within, 1024, 2),
-                  ID_S, k > 0);
+          mma_f16(d_s, sdesc(qa + atom * (kBM * 128) + within, 1024, 2),
+                  sdesc(ka + atom * (kBN * 128) + within, 1024, 2), ID_S, k > 0);
         }
-        mma_commit(&s_full[sb]);
+        mma_commit(&s_full[t]);
       }
       __syncwarp();
       return true;
     };
     auto issue_pv = [&](int j) -> bool {
       const uint32_t va = kv_addr + (j % kF16Stages) * L::STAGE_BYTES + L::K_BYTES;
-      for (int t = 0; t < 2; ++t) {
-        const int pb = 2 * t + (j & 1);
-        if (!warp_wait(&p_full[pb], (j >> 1) & 1, lim)) return false;
-        tc_fence_after();
-        const uint32_t pa = p_addr + pb * L::P_BYTES;
-        const uint32_t d = tmem + L::T_O + t * D;
-        if (elect_one()) {
+      if (!warp_wait(&p_full[t], j & 1, lim)) return false;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < kBN / 16; ++k)
-            mma_f16(d, sdesc(pa + 32 * k, 1024, 2), sdesc_lbo(va + 2048 * k, kBN * 128, 1024, 2), ID_PV,
-                    (j > 0 || k > 0) ? 1u : 0u);
-          mma_commit(&o_ready[t]);
-          mma_commit(&p_empty[pb]);
-          if (t == 1) mma_commit(&kv_empty[j % kF16Stages]);
+        for (int k = 0; k < kBN / 16; ++k) {
+          const uint64_t bd = sdesc_lbo(va + 2048 * k, kBN * 128, 1024, 2);
+          const uint32_t blo = static_cast<uint32_t>(bd), bhi = static_cast<uint32_t>(bd >> 32);
+          if (j == 0 && k == 0) mma_f16_ts<0>(d_o, ap + 8 * k, blo, bhi, ID_PV);
+          else mma_f16_ts<1>(d_o, ap + 8 * k, blo, bhi, ID_PV);
         }
-        __syncwarp();
+        mma_commit(&p_empty[t]);
+        mma_commit(&kv_empty[j % kF16Stages]);
       }
+      __syncwarp();
       return true;
     };
     for (int j = 0; ok && j < nkb; ++j) {
       if (!warp_wait(&kv_full[j % kF16Stages], (j / kF16Stages) & 1, lim)) { ok = false; break; }
       tc_fence_after();
-      if (!issue_s(j, 0) || !issue_s(j, 1)) { ok = false; break; }
+      if (!issue_s(j)) { ok = false; break; }
       if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
       if (warp_flag(sAbort)) { ok = false; break; }
     }
     if (ok) ok = issue_pv(nkb - 1);
     if (!ok && lane == 0) *sAbort = 1;
-    // every issued MMA completes before TMEM is released
-    if (elect_one()) mma_commit(mma_done);
+    // every MMA this warp issued completes before TMEM is released
+    if (elect_one()) mma_commit(&mma_done[t]);
     __syncwarp();
-    warp_wait(mma_done, 0, lim);
+    warp_wait(&mma_done[t], 0, lim);
   } else if (warp >= 4) {
     // ===================================================== query-tile warps
     const int t = (warp - 4) >> 2;       // tile 0 or 1
     const int r = tid & 127;             // row within the tile = TMEM lane
     const int row = q0 + t * kBM + r;
     const uint32_t t_lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS0 = tmem + L::T_S + 2 * t * kBN + t_lane;   // + (j & 1) * kBN
+    const uint32_t tS = tmem + L::T_S + t * kBN + t_lane;
+    const uint32_t tP = tmem + L::T_P + t * (kBN / 2) + t_lane;
     const uint32_t tO = tmem + L::T_O + t * D + t_lane;
     const float c = p.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     bool aborted = false;
 
     for (int j = 0; j < nkb; ++j) {
-      const int sb = 2 * t + (j & 1);
-      const uint32_t tS = tS0 + (j & 1) * kBN;
       const int nvalid = min(kBN, p.N - j * kBN);
-      if (!warp_wait(&s_full[sb], (j >> 1) & 1, lim)) { aborted = true; break; }
+      if (!warp_wait(&s_full[t], j & 1, lim)) { aborted = true; break; }
       tc_fence_after();
       uint32_t sr[kBN];
       {
@@ -249,10 +245,10 @@ __global__ void __launch_bounds__(kF16Threads, 1) attn_fp16_kernel(const __grid_
         tmem_ld32(tS + 32, s1);
         tmem_wait_dep2(s0, s1);
       }
-      // S is in registers: the MMA may overwrite this buffer with S(j+2)
+      // S is in registers: the MMA may compute S(j+1) into this buffer now
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[sb]);
+      if (lane == 0) mbar_arrive(&s_empty[t]);
       if (nvalid < kBN) {
 #pragma unroll
         for (int k = 0; k < kBN; ++k)
@@ -268,27 +264,14 @@ __global__ void __launch_bounds__(kF16Threads, 1) attn_fp16_kernel(const __grid_
       }
       const float m_blk = __fmul_rn(fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)), c);
 
-      // ---- raise the reference max (rare): rescale O (TMEM) and l ----
-      if (__any_sync(0xffffffffu, m_blk > m_ref + kRescaleLog2)) {
+      // ---- raise the reference max (rare); O is rescaled below ----
+      const bool raise = __any_sync(0xffffffffu, m_blk > m_ref + kRescaleLog2);
+      float alpha = 1.f;
+      if (raise) {
         const float m_new = fmaxf(m_ref, m_blk);
-        const float alpha = ex2_approx(m_ref - m_new);   // 0 while O is empty (m_ref = -inf)
+        alpha = ex2_approx(m_ref - m_new);   // 0 while O is empty (m_ref = -inf)
         m_ref = m_new;
         l *= alpha;
-        if (j > 0) {
-          // the previous block's P V has landed in O
-          if (!warp_wait(&o_ready[t], (j - 1) & 1, lim)) { aborted = true; break; }
-          tc_fence_after();
-#pragma unroll 1
-          for (int cb = 0; cb < D / 32; ++cb) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * cb, o);
-            tmem_wait_dep(o);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st32(tO + 32 * cb, o);
-          }
-          tmem_st_wait();
-        }
       }
 
       // ---- P = 2^(S c - m_ref) in fp16, row sum of the fp16 values in fp32 ----
@@ -306,21 +289,32 @@ __global__ void __launch_bounds__(kF16Threads, 1) attn_fp16_kernel(const __grid_
         pw[k / 2] = *reinterpret_cast<const uint32_t*>(&hp);
       }
       l += ls0 + ls1;
-      // the P V that read this buffer (block j - 2) has completed
-      if (j >= 2 && !warp_wait(&p_empty[sb], ((j >> 1) & 1) ^ 1, lim)) { aborted = true; break; }
-      uint8_t* sP = smem + L::OFF_P + sb * L::P_BYTES;
+      // the previous block's P V has completed: the P columns are free and O
+      // holds every block before this one
+      if (j > 0) {
+        if (!warp_wait(&p_empty[t], (j - 1) & 1, lim)) { aborted = true; break; }
+        tc_fence_after();
+        if (raise) {
+#pragma unroll 1
+          for (int cb = 0; cb < D / 32; ++cb) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * cb, o);
+            tmem_wait_dep(o);
 #pragma unroll
-      for (int k = 0; k < kBN / 8; ++k)
-        *reinterpret_cast<uint4*>(sP + swz<128>(r, 16 * k)) =
-            make_uint4(pw[4 * k], pw[4 * k + 1], pw[4 * k + 2], pw[4 * k + 3]);
-      fence_proxy_async_smem();
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st32(tO + 32 * cb, o);
+          }
+        }
+      }
+      tmem_st32(tP, pw);
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
+      if (lane == 0) mbar_arrive(&p_full[t]);
       if (warp_flag(sAbort)) { aborted = true; break; }
     }
     // ---- epilogue: out = O / l once the last P V has landed ----
-    if (!aborted && !warp_wait(&o_ready[t], (nkb - 1) & 1, lim)) aborted = true;
+    if (!aborted && !warp_wait(&p_empty[t], (nkb - 1) & 1, lim)) aborted = true;
     if (aborted) {
       *sAbort = 1;
     } else {
