@@ -131,6 +131,18 @@ def workload_config(w, l2_note):
 
 # ----------------------------------------------------------- CPU oracle ---
 
+# DRAM bytes (read + write) per attention launch, from one ncu capture of the
+# current kernels on the F = 3 sweep point (B=1, H=40, N=4680, profiles/), per
+# (head, token): the traffic is the K/V images or tiles and the output, linear
+# in B * heads * N.  None = no capture of the current kernel version.
+TRAFFIC_PER_HEAD_TOKEN = {"attn_int4_kernel": 1034.97, "attn_fp16_kernel": 1080.38}
+
+
+def traffic_per_launch(kernel, w, heads):
+    per = TRAFFIC_PER_HEAD_TOKEN.get(kernel)
+    return None if per is None or heads == 0 else per * w.B * heads * w.N
+
+
 def oracle_sample(w, q, k, v, rows: int = 128):
     """Time the CPU oracle on a bounded sample of the workload: the prologue of
     one head (all N tokens) and the INT4 attention of `rows` query rows of
@@ -303,12 +315,33 @@ def main():
     if rank == 0:
         ops = w.ops()
         value = ops * world / (ms_step * 1e-3) / 1e12
-        int8_peak = peaks["bf16"] * NOMINAL_INT8_PER_BF16
+        # The timed region is K back-to-back steps (well over a second of
+        # tensor-core load on the large configs), so the denominators are the
+        # sustained (power-capped) measured peaks; the burst ones ride along.
+        int8_peak = peaks["bf16_sus"] * NOMINAL_INT8_PER_BF16
+        int8_burst = peaks["bf16"] * NOMINAL_INT8_PER_BF16
         ms_int4 = statistics.mean(t_int4)
+        ms_f16 = statistics.mean(t_f16)
         ms_pro = statistics.mean(t_pro)
         n_int4_heads = int((flags == 0).sum())
         ops_int4 = 4.0 * w.B * n_int4_heads * w.N * w.N * w.d
-        achieved = ops_int4 / (ms_int4 * 1e-3) / 1e12 if n_int4_heads else 0.0
+        ops_f16 = 4.0 * w.B * int(flags.sum()) * w.N * w.N * w.d
+        if ms_int4 >= ms_f16:
+            kern, achieved = "attn_int4_kernel", (ops_int4 / (ms_int4 * 1e-3) / 1e12 if n_int4_heads else 0.0)
+            rl = {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": int8_peak,
+                  "unit": "TOPS (INT8 dense)", "frac": achieved / int8_peak,
+                  "peak_source": f"{peaks['source']} bf16 sustained {peaks['bf16_sus']} TFLOP/s x nominal INT8/BF16 "
+                                 f"ratio 2 (burst: {int8_burst:.1f}, frac {achieved / int8_burst:.3f})",
+                  "traffic": traffic_per_launch(kern, w, n_int4_heads), "algorithmic_ops_per_launch": ops_int4,
+                  "int8_spec_frac": achieved / INT8_SPEC_TOPS}
+        else:
+            kern = "attn_fp16_kernel"
+            achieved = ops_f16 / (ms_f16 * 1e-3) / 1e12
+            rl = {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sus"],
+                  "unit": "TFLOP/s (FP16/BF16 dense)", "frac": achieved / peaks["bf16_sus"],
+                  "peak_source": f"{peaks['source']} bf16 sustained {peaks['bf16_sus']} TFLOP/s "
+                                 f"(burst: {peaks['bf16']}, frac {achieved / peaks['bf16']:.3f})",
+                  "traffic": traffic_per_launch(kern, w, int(flags.sum())), "algorithmic_ops_per_launch": ops_f16}
         # prologue algorithmic bytes: fp16 Q,K,V read; packed codes + scales written
         nblk = (w.N + 63) // 64
         pro_bytes = w.B * w.H * (3 * w.N * w.d * 2 + 3 * nblk * 64 * w.d // 2 + 2 * nblk * 4 + nblk * w.d * 4)
@@ -322,13 +355,9 @@ def main():
             "config": workload_config(w, "inputs > L2: fp16 Q/K/V %.2f GB, INT4 codes %.2f GB per step, no flush"
                                       % (3 * q.nbytes / 1e9, 3 * w.B * w.H * nblk * 64 * w.d / 2 / 1e9)),
             "pct_int8_spec": 100.0 * value / world / INT8_SPEC_TOPS,
-            "breakdown_ms": {"prologue": ms_pro, "int4_attention": ms_int4, "fp16_fallback": statistics.mean(t_f16)},
+            "breakdown_ms": {"prologue": ms_pro, "int4_attention": ms_int4, "fp16_fallback": ms_f16},
             "prologue_gbs": pro_bytes / (ms_pro * 1e-3) / 1e9,
-            "roofline": {"kernel": "attn_int4_kernel", "bound": "tensor", "achieved": achieved,
-                         "peak": int8_peak, "unit": "TOPS (INT8 dense)", "frac": achieved / int8_peak,
-                         "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} TFLOP/s x nominal INT8/BF16 ratio 2",
-                         "traffic": None, "algorithmic_ops_per_launch": ops_int4,
-                         "int8_spec_frac": achieved / INT8_SPEC_TOPS},
+            "roofline": rl,
             "e2e": {"value": ops * world / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
             "gpu_launches": launches_per_step * args.steps,
