@@ -33,7 +33,7 @@
 //
 // One CTA = two 128-row query tiles of one head (256 rows), 384 threads:
 //   warp 0      TMA producer: the K, V'_hi and V'_lo tiles of each 64-key
-//               block -> a 3-stage shared-memory ring (cp.async.bulk);
+//               block -> a 4-stage shared-memory ring (cp.async.bulk);
 //   warps 1, 2  MMA issuers of tile 0 and tile 1 (warp-uniform loops, one
 //               elected lane issues); warp 1 also owns the TMEM allocation;
 //   warp 3      idle;
@@ -77,7 +77,7 @@ struct Int4Params {
 
 constexpr int kInt4Threads = 384;
 constexpr int kRowsPerCta = 2 * kBM;
-constexpr int kOps = 3;   // operand stages
+constexpr int kOps = 4;   // operand stages
 constexpr int kProducerRegs = 40;
 constexpr int kConsumerRegs = 232;
 // Register split: kProducerRegs * 128 + kConsumerRegs * 256 equals the launch
@@ -98,9 +98,9 @@ struct Int4Smem {
   static constexpr int OFF_OP = 0;                                // kOps stages
   static constexpr int OFF_TAU = OFF_OP + kOps * OP_BYTES;
   static constexpr int OFF_BAR = OFF_TAU + 64;
-  // barriers: op_full[3] op_empty[3] s_full[2 tiles] s_empty[2] p_full[2]
+  // barriers: op_full[kOps] op_empty[kOps] s_full[2 tiles] s_empty[2] p_full[2]
   //           p_empty[2] q_full mma_done[2]
-  static constexpr int NBAR = 3 + 3 + 2 + 2 + 2 + 2 + 1 + 2;
+  static constexpr int NBAR = 2 * kOps + 2 + 2 + 2 + 2 + 1 + 2;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int BYTES = OFF_ABORT + 4;
@@ -164,16 +164,16 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* op_full = bars;
-  uint64_t* op_empty = bars + 3;
+  uint64_t* op_empty = bars + kOps;
   // per tile, once per block (phase j & 1)
-  uint64_t* s_full = bars + 6;
-  uint64_t* s_empty = bars + 8;
-  uint64_t* p_full = bars + 10;
+  uint64_t* s_full = bars + 2 * kOps;
+  uint64_t* s_empty = bars + 2 * kOps + 2;
+  uint64_t* p_full = bars + 2 * kOps + 4;
   // p_empty[t]: tile t's P V of the block has completed -- the P columns may
   // be rewritten, and O holds every block up to that one
-  uint64_t* p_empty = bars + 12;
-  uint64_t* q_full = bars + 14;
-  uint64_t* mma_done = bars + 15;   // [2], one per MMA warp
+  uint64_t* p_empty = bars + 2 * kOps + 6;
+  uint64_t* q_full = bars + 2 * kOps + 8;
+  uint64_t* mma_done = bars + 2 * kOps + 9;   // [2], one per MMA warp
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + L::OFF_ABORT);
   float* sTau = reinterpret_cast<float*>(smem + L::OFF_TAU);
