@@ -188,7 +188,7 @@ __device__ __forceinline__ void load_tile(const __half* src, int n0, int N, floa
 }
 
 template <int D>
-__global__ void __launch_bounds__(kPrologueThreads, 4) prologue_kernel(const PrologueParams p) {
+__global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const PrologueParams p) {
   constexpr int LD = D + 1;
   __shared__ float X[64 * LD];
   __shared__ float red[kPrologueThreads / 32];
