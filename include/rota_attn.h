@@ -78,11 +78,14 @@ typedef struct {
  *                      (may be NULL when no head is flagged)
  *   rope_cos, rope_sin: fp32 tables from rota_attn_build_rope_tables, copied
  *                      to the device by the caller.
- *   int4_work        : workspace of rota_attn_fwd_int4 (bytes[ROTA_BUF_INT4_WORK]):
- *                      the K and V codes of the INT4 heads widened once per call
- *                      into the 8-bit tensor-core operand tiles (pre-swizzled
- *                      e4m3 images) and the V scales times 2^9.  Transient: its
- *                      contents are rewritten by every call.
+ *   int4_work        : workspace of rota_attn_fwd_int4 (bytes[ROTA_BUF_INT4_WORK],
+ *                      320 * head_dim bytes per (head, 64-key block)): the K
+ *                      and V codes of the INT4 heads widened once per call into
+ *                      pre-swizzled tensor-core operand images -- K as e4m3
+ *                      (64 x head_dim), V with its channel scale folded in as
+ *                      two exact fp16 tiles v * s_hi and v * s_lo (head_dim x 64
+ *                      each).  Transient: its contents are rewritten by every
+ *                      call.
  */
 typedef struct {
   uint8_t* q_codes;

@@ -35,7 +35,10 @@ struct PrologueParams {
   int grid_h, grid_w;
   int rope_dim[3];
   int had[3];
-  int unit[3];       // channels per rotation unit: max(2, had[a])
+  int fused[3];      // partition a is rotated in registers while the tile is loaded
+                     // (no rotation, or had[a] <= 8 and coff[a] % had[a] == 0: every
+                     // unit then lies inside one 8-channel chunk)
+  int any_unfused;   // some partition needs the shared-memory rotation pass
   int coff[3];       // channel offset of each partition
   int toff[3];       // table offset of each axis
   float rnorm[3];    // RN(1 / sqrt(had[a]))
@@ -64,65 +67,56 @@ __device__ __forceinline__ void rope_pair(float& x0, float& x1, float c, float s
   x1 = __fadd_rn(a1, b1);
 }
 
-// One rotation unit of G channels of one token held in the smem row: RoPE on
-// its G/2 pairs, then (if rot) the Walsh-Hadamard butterflies h = 1..G/2 and
-// the normalisation.  Returns the unit's max |y|.
+// Walsh-Hadamard butterflies h = 1..G/2 and the normalisation of one rotation
+// unit of G channels whose RoPE has been applied already, in place in the smem
+// row.  Returns the unit's max |y|.
 template <int G>
-__device__ __forceinline__ float rope_rotate_unit(float* xrow, int c0, int pair0, const float* ct,
-                                                  const float* st, bool rot, float rnorm) {
+__device__ __forceinline__ float rotate_unit(float* xrow, int c0, float rnorm) {
   float y[G];
 #pragma unroll
   for (int j = 0; j < G; ++j) y[j] = xrow[c0 + j];
 #pragma unroll
-  for (int j = 0; j < G / 2; ++j) {
-    rope_pair(y[2 * j], y[2 * j + 1], __ldg(ct + pair0 + j), __ldg(st + pair0 + j));
-  }
-  if (rot) {
+  for (int h = 1; h < G; h <<= 1) {
 #pragma unroll
-    for (int h = 1; h < G; h <<= 1) {
-#pragma unroll
-      for (int j = 0; j < G; ++j) {
-        if (j & h) continue;
-        const float u = y[j], w = y[j + h];
-        y[j] = __fadd_rn(u, w);
-        y[j + h] = __fsub_rn(u, w);
-      }
+    for (int j = 0; j < G; ++j) {
+      if (j & h) continue;
+      const float u = y[j], w = y[j + h];
+      y[j] = __fadd_rn(u, w);
+      y[j + h] = __fsub_rn(u, w);
     }
-#pragma unroll
-    for (int j = 0; j < G; ++j) y[j] = __fmul_rn(y[j], rnorm);
   }
   float amax = 0.f;
 #pragma unroll
   for (int j = 0; j < G; ++j) {
+    y[j] = __fmul_rn(y[j], rnorm);
     xrow[c0 + j] = y[j];
     amax = fmaxf(amax, fabsf(y[j]));
   }
   return amax;
 }
 
-// The same unit for G >= 16, in place in the smem row (no register arrays).
-__device__ __noinline__ float rope_rotate_unit_smem(float* xrow, int c0, int G, int pair0, const float* ct,
-                                                   const float* st, bool rot, float rnorm) {
+__device__ __noinline__ float rotate_unit_smem(float* xrow, int c0, int G, float rnorm) {
   float* y = xrow + c0;
-  for (int j = 0; j < G / 2; ++j) {
-    float x0 = y[2 * j], x1 = y[2 * j + 1];
-    rope_pair(x0, x1, __ldg(ct + pair0 + j), __ldg(st + pair0 + j));
-    y[2 * j] = x0;
-    y[2 * j + 1] = x1;
-  }
-  if (rot) {
-    for (int h = 1; h < G; h <<= 1)
-      for (int j = 0; j < G; ++j) {
-        if (j & h) continue;
-        const float u = y[j], w = y[j + h];
-        y[j] = __fadd_rn(u, w);
-        y[j + h] = __fsub_rn(u, w);
-      }
-    for (int j = 0; j < G; ++j) y[j] = __fmul_rn(y[j], rnorm);
-  }
+  for (int h = 1; h < G; h <<= 1)
+    for (int j = 0; j < G; ++j) {
+      if (j & h) continue;
+      const float u = y[j], w = y[j + h];
+      y[j] = __fadd_rn(u, w);
+      y[j + h] = __fsub_rn(u, w);
+    }
   float amax = 0.f;
-  for (int j = 0; j < G; ++j) amax = fmaxf(amax, fabsf(y[j]));
+  for (int j = 0; j < G; ++j) {
+    y[j] = __fmul_rn(y[j], rnorm);
+    amax = fmaxf(amax, fabsf(y[j]));
+  }
   return amax;
+}
+
+// One butterfly (u, w) -> (u + w, u - w) where `on`, else unchanged.
+__device__ __forceinline__ void bfly(float& u, float& w, bool on) {
+  const float s = __fadd_rn(u, w), d = __fsub_rn(u, w);
+  u = on ? s : u;
+  w = on ? d : w;
 }
 
 __device__ __forceinline__ float block_max(float v, float* red) {
@@ -141,28 +135,31 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return red[0];
 }
 
-__device__ __forceinline__ int quant_code(float y, float inv) {
-  const int c = __float2int_rn(__fmul_rn(y, inv));  // round half to even
-  return max(-7, min(7, c));
+// Sign-magnitude nibble of the code of y: c = RNE_int(RN(y * inv)) by adding
+// 1.5 * 2^23 (the sum's integer part is the round-half-even integer of any
+// |f| < 2^22).  |y| <= amax and inv = RN(7 / amax) bound |f| by 7 (1 + 2^-24),
+// which rounds to at most 7: no clamp is needed.
+__device__ __forceinline__ uint32_t code_nibble(float y, float inv) {
+  const float f = __fmul_rn(y, inv);
+  const int c = __float_as_int(__fadd_rn(f, 12582912.f)) - 0x4B400000;
+  return static_cast<uint32_t>(abs(c)) | ((static_cast<uint32_t>(c) >> 28) & 8u);
 }
 
-// Sign-magnitude nibble of a code in [-7, 7]: bit 3 = sign, bits 0-2 = |v|.
-__device__ __forceinline__ uint32_t nibble(int c) { return static_cast<uint32_t>(c < 0 ? 8 - c : c); }
-
-// Eight codes -> one packed word: byte j holds element j (low nibble) and j+4 (high).
-__device__ __forceinline__ uint32_t pack8(const int (&c)[8]) {
-  uint32_t w = 0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) w |= (nibble(c[j]) | (nibble(c[j + 4]) << 4)) << (8 * j);
-  return w;
+// Codes of elements 0-3 (a) and 4-7 (b) -> one packed word (byte j: element j
+// low, element j + 4 high).
+__device__ __forceinline__ uint32_t pack8_f(float4 a, float4 b, float inv) {
+  return (code_nibble(a.x, inv) | (code_nibble(b.x, inv) << 4)) |
+         ((code_nibble(a.y, inv) | (code_nibble(b.y, inv) << 4)) << 8) |
+         ((code_nibble(a.z, inv) | (code_nibble(b.z, inv) << 4)) << 16) |
+         ((code_nibble(a.w, inv) | (code_nibble(b.w, inv) << 4)) << 24);
 }
 
-// fp16 tile [64, D] of one (head, block) -> fp32 smem rows of stride D+1.
-// Every thread issues all of its 16-byte loads before it converts any, so a
-// CTA waits for one memory latency rather than one per load.
+// fp16 tile [64, D] of one (head, block) -> fp32 smem rows of stride D + 4
+// (16-byte aligned rows).  Every thread issues all of its 16-byte loads before
+// it converts any, so a CTA waits for one memory latency rather than one per load.
 template <int D>
 __device__ __forceinline__ void load_tile(const __half* src, int n0, int N, float* X) {
-  constexpr int LD = D + 1;
+  constexpr int LD = D + 4;
   constexpr int PER = 64 * D / 8 / kPrologueThreads;
   static_assert(PER * kPrologueThreads * 8 == 64 * D, "tile split");
   uint4 u[PER];
@@ -178,20 +175,20 @@ __device__ __forceinline__ void load_tile(const __half* src, int n0, int N, floa
     const int i = threadIdx.x + k * kPrologueThreads;
     const int r = i / (D / 8), ch = i % (D / 8);
     const __half2* h2 = reinterpret_cast<const __half2*>(&u[k]);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 t = __half22float2(h2[j]);
-      X[r * LD + ch * 8 + 2 * j] = t.x;
-      X[r * LD + ch * 8 + 2 * j + 1] = t.y;
-    }
+    const float2 t0 = __half22float2(h2[0]), t1 = __half22float2(h2[1]);
+    const float2 t2 = __half22float2(h2[2]), t3 = __half22float2(h2[3]);
+    float4* xr = reinterpret_cast<float4*>(X + r * LD + ch * 8);
+    xr[0] = make_float4(t0.x, t0.y, t1.x, t1.y);
+    xr[1] = make_float4(t2.x, t2.y, t3.x, t3.y);
   }
 }
 
 template <int D>
 __global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const PrologueParams p) {
-  constexpr int LD = D + 1;
-  __shared__ float X[64 * LD];
+  constexpr int LD = D + 4;
+  __shared__ __align__(16) float X[64 * LD];
   __shared__ float red[kPrologueThreads / 32];
+  __shared__ int4 sPos[64];
 
   const int blk = blockIdx.x, h = blockIdx.y;
   const int b = blockIdx.z / 3, which = blockIdx.z % 3;
@@ -227,65 +224,135 @@ __global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const Pro
       }
       return;
     }
-    load_tile<D>(src, n0, p.N, X);
-    __syncthreads();
-
-    // RoPE + rotation, one (partition, unit, token) job per iteration, tokens fastest.
-    float amax = 0.f;
-    int pos_cache_n = -1;
-    int pos[3] = {0, 0, 0};
-    int jbase = 0;
-#pragma unroll 1
-    for (int a = 0; a < 3; ++a) {
-      const int G = p.unit[a];
-      const int nunits = p.rope_dim[a] / G;
-      const int njobs = 64 * nunits;
-      const int half = p.rope_dim[a] >> 1;
-      const bool rot = p.had[a] > 1;
-#pragma unroll 1
-      for (int j = threadIdx.x; j < njobs; j += kPrologueThreads) {
-        const int r = j & 63, u = j >> 6;
-        const int n = n0 + r;
-        if (n >= p.N) continue;
-        if (n != pos_cache_n) {
-          token_pos(p, n, pos);
-          pos_cache_n = n;
-        }
-        float* xrow = X + r * LD;
-        const int c0 = p.coff[a] + u * G;
-        const float* ct = p.cos_tab + p.toff[a] + pos[a] * half;
-        const float* st = p.sin_tab + p.toff[a] + pos[a] * half;
-        const int pair0 = (u * G) >> 1;
-        float m;
-        switch (G) {
-          case 2: m = rope_rotate_unit<2>(xrow, c0, pair0, ct, st, rot, p.rnorm[a]); break;
-          case 4: m = rope_rotate_unit<4>(xrow, c0, pair0, ct, st, rot, p.rnorm[a]); break;
-          case 8: m = rope_rotate_unit<8>(xrow, c0, pair0, ct, st, rot, p.rnorm[a]); break;
-          default: m = rope_rotate_unit_smem(xrow, c0, G, pair0, ct, st, rot, p.rnorm[a]); break;
-        }
-        amax = fmaxf(amax, m);
-      }
-      jbase += njobs;
+    // Each thread owns one 8-channel chunk ch of rows rb, rb + RSTEP, ...: RoPE
+    // pairs never straddle a chunk, nor do the rotation units of the fused
+    // partitions, so both are applied in registers before the row is stored.
+    constexpr int CH = D / 8;
+    constexpr int RSTEP = kPrologueThreads / CH;
+    constexpr int PER = 64 / RSTEP;
+    static_assert(CH * RSTEP == kPrologueThreads && PER * RSTEP == 64, "tile split");
+    const int ch = threadIdx.x % CH, rb = threadIdx.x / CH;
+    uint4 u[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int n = n0 + rb + k * RSTEP;
+      u[k] = n < p.N ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)n * D + ch * 8)) : make_uint4(0, 0, 0, 0);
     }
-    (void)jbase;
+    // token coordinates of the block's tokens, while the loads are in flight
+    if (threadIdx.x < 64) {
+      int pos[3];
+      token_pos(p, n0 + threadIdx.x, pos);
+      sPos[threadIdx.x] = make_int4(pos[0], pos[1], pos[2], 0);
+    }
+    // the chunk's four RoPE pairs: axis, table row base, rotation levels, norm
+    int ax[4], tb[4], hf[4];
+    float rn[4];
+    bool l1[4], l2[4], fz[4];
+    bool l3 = false, any2 = false;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int c = ch * 8 + 2 * q;
+      const int a = c < p.coff[1] ? 0 : (c < p.coff[2] ? 1 : 2);
+      const int G = p.had[a];
+      ax[q] = a;
+      tb[q] = p.toff[a] + ((c - p.coff[a]) >> 1);
+      hf[q] = p.rope_dim[a] >> 1;
+      fz[q] = p.fused[a] != 0;
+      const bool rot = fz[q] && G > 1;
+      l1[q] = rot;
+      l2[q] = rot && G >= 4;
+      if (q == 0) l3 = rot && G >= 8;
+      any2 = any2 || l2[q];
+      rn[q] = rot ? p.rnorm[a] : 1.f;
+    }
+    any2 = __any_sync(0xffffffffu, any2);
+    const bool any3 = __any_sync(0xffffffffu, l3);
+    __syncthreads();   // sPos
+
+    float amax = 0.f;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int r = rb + k * RSTEP;
+      float y[8];
+      {
+        const __half2* h2 = reinterpret_cast<const __half2*>(&u[k]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 t = __half22float2(h2[j]);
+          y[2 * j] = t.x;
+          y[2 * j + 1] = t.y;
+        }
+      }
+      if (n0 + r < p.N) {
+        const int4 ps = sPos[r];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int pa = ax[q] == 0 ? ps.x : (ax[q] == 1 ? ps.y : ps.z);
+          const int ti = tb[q] + pa * hf[q];
+          rope_pair(y[2 * q], y[2 * q + 1], __ldg(p.cos_tab + ti), __ldg(p.sin_tab + ti));
+        }
+        // Walsh-Hadamard levels h = 1, 2, 4 inside the units of the fused partitions
+#pragma unroll
+        for (int q = 0; q < 4; ++q) bfly(y[2 * q], y[2 * q + 1], l1[q]);
+        if (any2) {
+          bfly(y[0], y[2], l2[0]);
+          bfly(y[1], y[3], l2[0]);
+          bfly(y[4], y[6], l2[2]);
+          bfly(y[5], y[7], l2[2]);
+        }
+        if (any3) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) bfly(y[j], y[j + 4], l3);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          y[j] = __fmul_rn(y[j], rn[j >> 1]);
+          if (fz[j >> 1]) amax = fmaxf(amax, fabsf(y[j]));
+        }
+      }
+      float4* xr = reinterpret_cast<float4*>(X + r * LD + ch * 8);
+      xr[0] = make_float4(y[0], y[1], y[2], y[3]);
+      xr[1] = make_float4(y[4], y[5], y[6], y[7]);
+    }
+
+    // the other partitions' rotation units, (partition, unit, token) jobs in smem
+    if (p.any_unfused) {
+      __syncthreads();
+#pragma unroll 1
+      for (int a = 0; a < 3; ++a) {
+        if (p.fused[a]) continue;
+        const int G = p.had[a];
+        const int njobs = 64 * (p.rope_dim[a] / G);
+#pragma unroll 1
+        for (int j = threadIdx.x; j < njobs; j += kPrologueThreads) {
+          const int r = j & 63, un = j >> 6;
+          if (n0 + r >= p.N) continue;
+          float* xrow = X + r * LD;
+          const int c0 = p.coff[a] + un * G;
+          float m;
+          switch (G) {
+            case 2: m = rotate_unit<2>(xrow, c0, p.rnorm[a]); break;
+            case 4: m = rotate_unit<4>(xrow, c0, p.rnorm[a]); break;
+            case 8: m = rotate_unit<8>(xrow, c0, p.rnorm[a]); break;
+            default: m = rotate_unit_smem(xrow, c0, G, p.rnorm[a]); break;
+          }
+          amax = fmaxf(amax, m);
+        }
+      }
+    }
     amax = block_max(amax, red);  // includes the __syncthreads that publishes X
     const float scale = amax == 0.f ? 0.f : __fdiv_rn(amax, 7.f);
     const float inv = amax == 0.f ? 0.f : __fdiv_rn(7.f, amax);
     uint8_t* cdst = (which == 0 ? p.q_codes : p.k_codes) + (head * npad + n0) * (D / 2);
     for (int i = threadIdx.x; i < 64 * D / 16; i += kPrologueThreads) {
-      const int r = i & 63, ch = i >> 6;  // 16 channels -> 8 bytes
-      const float* xr = X + r * LD + ch * 16;
-      uint32_t w[2] = {0u, 0u};
+      const int r = i & 63, g = i >> 6;  // 16 channels -> 8 bytes
+      uint2 w = make_uint2(0u, 0u);
       if (n0 + r < p.N) {
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          int c[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) c[j] = quant_code(xr[8 * g + j], inv);
-          w[g] = pack8(c);
-        }
+        const float4* xr = reinterpret_cast<const float4*>(X + r * LD + g * 16);
+        const float4 v0 = xr[0], v1 = xr[1], v2 = xr[2], v3 = xr[3];
+        w = make_uint2(pack8_f(v0, v1, inv), pack8_f(v2, v3, inv));
       }
-      *reinterpret_cast<uint2*>(cdst + (size_t)r * (D / 2) + ch * 8) = make_uint2(w[0], w[1]);
+      *reinterpret_cast<uint2*>(cdst + (size_t)r * (D / 2) + g * 8) = w;
     }
     if (threadIdx.x == 0) (which == 0 ? p.q_scale : p.k_scale)[head * p.nblk + blk] = scale;
     return;
@@ -312,13 +379,14 @@ __global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const Pro
     uint32_t w[RPT / 8];
 #pragma unroll
     for (int j = 0; j < RPT / 8; ++j) {
-      int cs[8];
+      uint32_t wj = 0u;
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
         const int r = r0 + 8 * j + t;
-        cs[t] = (n0 + r < p.N) ? quant_code(X[r * LD + c], inv) : 0;
+        const uint32_t nb = (n0 + r < p.N) ? code_nibble(X[r * LD + c], inv) : 0u;
+        wj |= nb << (t < 4 ? 8 * t : 8 * (t - 4) + 4);
       }
-      w[j] = pack8(cs);
+      w[j] = wj;
     }
     uint32_t* dst = reinterpret_cast<uint32_t*>(p.v_codes + ((head * p.nblk + blk) * D + c) * 32) + part * (RPT / 8);
 #pragma unroll

@@ -272,10 +272,11 @@ rota_status rota_attn_prepare_qk(const rota_attn_desc* d, const uint16_t* q, con
   for (int a = 0; a < 3; ++a) {
     p.rope_dim[a] = d->rope_dim[a];
     p.had[a] = d->had_block[a];
-    p.unit[a] = d->had_block[a] < 2 ? 2 : d->had_block[a];
     p.coff[a] = coff;
     p.toff[a] = toff;
     p.rnorm[a] = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d->had_block[a])));
+    p.fused[a] = d->had_block[a] <= 1 || (d->had_block[a] <= 8 && coff % d->had_block[a] == 0);
+    if (!p.fused[a]) p.any_unfused = 1;
     coff += d->rope_dim[a];
     toff += extent[a] * (d->rope_dim[a] / 2);
   }
