@@ -206,6 +206,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=128)      # per step of --impl reference
     ap.add_argument("--cpu-rows", type=int, default=1024)     # the cpu_baseline sample (about 10 s)
+    ap.add_argument("--chunk-heads", type=int, default=0)     # heads per chunk of the e2e pipeline (0: library default)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -288,18 +289,18 @@ def main():
     t_f16 = [e[2].elapsed_time(e[3]) for e in evs]
 
     # end to end through the public API: pinned host inputs in, fp32 output back, every step
+    # (rota_attn_forward_host: head chunks, copies of neighbouring chunks overlapping the kernels)
     e2e_steps = max(3, min(args.steps, 10))
+    chunk_heads = args.chunk_heads or ra.rota_attn_pipeline_chunk_heads(
+        att.desc, torch.cuda.get_device_properties(dev).multi_processor_count)
+    att.forward_host(qh, kh, vh, flags, out_h, heads_per_chunk=chunk_heads, stream=stream)   # staging, warm-up
     barrier()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        att.forward(qd, kd, vd, flags, out)
-        out_h.copy_(out, non_blocking=True)
+        att.forward_host(qh, kh, vh, flags, out_h, heads_per_chunk=chunk_heads, stream=stream)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -359,7 +360,8 @@ def main():
             "prologue_gbs": pro_bytes / (ms_pro * 1e-3) / 1e9,
             "roofline": rl,
             "e2e": {"value": ops * world / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+                    "heads_per_chunk": chunk_heads},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }

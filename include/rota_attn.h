@@ -13,7 +13,9 @@
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers allocated by the caller, except
  *     where a parameter is marked "host".  The library never allocates,
- *     never frees and never synchronises (except rota_attn_get_error).
+ *     never frees and never synchronises (except rota_attn_get_error), apart
+ *     from the copy streams and events that rota_attn_pipeline_create makes
+ *     on request and rota_attn_pipeline_destroy releases.
  *   - fp16 tensors are passed as their uint16_t bit patterns.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream); every
  *     device call is enqueued asynchronously on it.
@@ -69,7 +71,7 @@ typedef struct {
 /*
  * Caller-owned device buffers written by rota_attn_prepare_qk and read by the
  * attention calls (sizes from rota_attn_buffer_sizes; every pointer 16-byte
- * aligned):
+ * aligned, except q_scale and k_scale, which need 4 bytes):
  *   q_codes, k_codes : uint8 [B,H,Npad,head_dim/2]  rotated, RoPE'd Q/K codes
  *   q_scale, k_scale : fp32  [B,H,nblk]               one scale per 64 tokens
  *   v_codes          : uint8 [B,H,nblk,head_dim,32]  64 tokens of one channel
@@ -177,6 +179,50 @@ rota_status rota_attn_fwd_int4(const rota_attn_desc* desc, const rota_attn_buffe
 rota_status rota_attn_fwd_fp16_fallback(const rota_attn_desc* desc, const rota_attn_buffers* buf,
                                         const uint16_t* v, const uint8_t* head_flags, float* out,
                                         void* stream);
+
+/*
+ * Host-to-host forward (a packaging of the three calls above for inputs that
+ * live in host memory; the paper has no counterpart).  q_host, k_host,
+ * v_host: host fp16 [B,H,N,head_dim]; out_host: host fp32 [B,H,N,head_dim];
+ * pinned (page-locked) host memory is needed for the copies to overlap the
+ * kernels.  q_dev, k_dev, v_dev, out_dev: caller-owned device buffers of the
+ * same shapes (16-byte aligned), used as staging; buf and head_flags as for
+ * rota_attn_prepare_qk / rota_attn_fwd_int4 / rota_attn_fwd_fp16_fallback.
+ *
+ * The heads of each batch entry are taken in chunks of heads_per_chunk
+ * (0 = rota_attn_pipeline_chunk_heads for this device): chunk c's inputs are
+ * copied in on the pipeline's host-to-device stream, its prologue, INT4
+ * attention and FP16 fallback run on `stream`, and its output is copied out
+ * on the device-to-host stream, so the copies of neighbouring chunks overlap
+ * chunk c's kernels.  Every result is the one the three calls give on the
+ * whole problem (heads are independent).  Ordering: the copies start after
+ * the work already enqueued on `stream`, and `stream` continues only after
+ * the last copy-out, so out_host is complete once `stream` has reached that
+ * point (e.g. after rota_attn_get_error(stream)).  Neither host buffer may be
+ * touched by the caller until then.  Errors: ROTA_ERR_INVALID_ARG for a null
+ * pointer, a negative heads_per_chunk or a pipeline made on another device;
+ * ROTA_ERR_UNSUPPORTED if the pipeline has too few events (2 per chunk + 2);
+ * otherwise the first failing call's status (the streams are still joined).
+ */
+typedef struct rota_attn_pipeline rota_attn_pipeline;
+
+/* Creates, on the current device, the two copy streams (non-blocking) and the
+ * events for up to max_chunks chunks per call.  *out receives the handle. */
+rota_status rota_attn_pipeline_create(int32_t max_chunks, rota_attn_pipeline** out);
+
+/* Releases what rota_attn_pipeline_create made (NULL is a no-op). */
+rota_status rota_attn_pipeline_destroy(rota_attn_pipeline* pipeline);
+
+/* The default chunk size: heads per chunk that minimise the waves of the
+ * attention kernel over all chunks plus the unhidden copies of the first and
+ * last chunk, for a device with num_sms SMs (0 on an invalid descriptor). */
+int32_t rota_attn_pipeline_chunk_heads(const rota_attn_desc* desc, int32_t num_sms);
+
+rota_status rota_attn_forward_host(const rota_attn_desc* desc, const uint16_t* q_host, const uint16_t* k_host,
+                                   const uint16_t* v_host, const uint8_t* head_flags, float* out_host,
+                                   uint16_t* q_dev, uint16_t* k_dev, uint16_t* v_dev, float* out_dev,
+                                   const rota_attn_buffers* buf, int32_t heads_per_chunk,
+                                   rota_attn_pipeline* pipeline, void* stream);
 
 /* Synchronises `stream`, then returns and clears the device error word
  * (ROTA_OK, ROTA_ERR_TIMEOUT or ROTA_ERR_DEVICE), or ROTA_ERR_CUDA if the

@@ -249,6 +249,13 @@ __global__ void __launch_bounds__(kF16Threads, 1) attn_fp16_kernel(const __grid_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[t]);
+      // Rows past N hold whatever follows the head in the Q view; their scores
+      // are taken as 0, so that the warp's vote on raising the reference max
+      // (which every row of the warp follows) depends on valid rows only.
+      if (row >= p.N) {
+#pragma unroll
+        for (int k = 0; k < kBN; ++k) sr[k] = 0u;
+      }
       if (nvalid < kBN) {
 #pragma unroll
         for (int k = 0; k < kBN; ++k)

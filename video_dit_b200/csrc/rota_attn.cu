@@ -6,6 +6,10 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <new>
+#include <type_traits>
+#include <vector>
+#include <algorithm>
 
 #include <cuda_runtime.h>
 
@@ -73,6 +77,17 @@ rota_status set_smem(K kernel, int bytes) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// The buffers the INT4 path reads or writes: q_scale and k_scale are touched
+// one float at a time (4-byte alignment), the others with 16-byte accesses.
+bool int4_buffers_ok(const rota_attn_buffers* buf, bool with_work) {
+  const void* v16[] = {buf->q_codes, buf->k_codes, buf->v_codes, buf->v_scale};
+  for (const void* ptr : v16)
+    if (!ptr || !aligned16(ptr)) return false;
+  if (!buf->q_scale || !buf->k_scale || !aligned4(buf->q_scale) || !aligned4(buf->k_scale)) return false;
+  return !with_work || (buf->int4_work && aligned16(buf->int4_work));
+}
 
 // Heads with flag == want, written to `heads`; returns their count.
 int select_heads(const rota_attn_desc* d, const uint8_t* flags, int want, int16_t* heads) {
@@ -240,11 +255,7 @@ rota_status rota_attn_prepare_qk(const rota_attn_desc* d, const uint16_t* q, con
   int16_t tmp[256];
   const int n_int4 = select_heads(d, head_flags, 0, tmp);
   const int n_fp16 = d->H - n_int4;
-  if (n_int4 > 0) {
-    const void* need[] = {buf->q_codes, buf->k_codes, buf->q_scale, buf->k_scale, buf->v_codes, buf->v_scale};
-    for (const void* ptr : need)
-      if (!ptr || !aligned16(ptr)) return ROTA_ERR_INVALID_ARG;
-  }
+  if (n_int4 > 0 && !int4_buffers_ok(buf, false)) return ROTA_ERR_INVALID_ARG;
   if (n_fp16 > 0 && (!buf->q_rope || !buf->k_rope || !aligned16(buf->q_rope) || !aligned16(buf->k_rope)))
     return ROTA_ERR_INVALID_ARG;
 
@@ -298,10 +309,7 @@ static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers*
   rota_status st = rota_attn_validate(d);
   if (st != ROTA_OK) return st;
   if (!buf || !out || !aligned16(out)) return ROTA_ERR_INVALID_ARG;
-  const void* need[] = {buf->q_codes, buf->k_codes, buf->q_scale, buf->k_scale, buf->v_codes, buf->v_scale,
-                        buf->int4_work};
-  for (const void* ptr : need)
-    if (!ptr || !aligned16(ptr)) return ROTA_ERR_INVALID_ARG;
+  if (!int4_buffers_ok(buf, true)) return ROTA_ERR_INVALID_ARG;
 
   static rota::Int4Params p;  // large (heads list); filled under a lock below
   static std::mutex mu;
@@ -406,6 +414,167 @@ rota_status rota_attn_fwd_fp16_fallback(const rota_attn_desc* d, const rota_attn
   const dim3 grid((d->N + 2 * rota::kBM - 1) / (2 * rota::kBM), p.nheads, d->B);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d->head_dim == 128 ? launch_fp16_kernel<128>(p, grid, s) : launch_fp16_kernel<64>(p, grid, s);
+}
+
+// ---------------------------------------------------------------------------
+// Host-to-host forward: the heads are processed in chunks, with the copies of
+// the neighbouring chunks on two copy streams while a chunk computes.
+// ---------------------------------------------------------------------------
+struct rota_attn_pipeline {
+  int device = 0;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  std::vector<cudaEvent_t> events;   // 2 per chunk + 2
+};
+
+rota_status rota_attn_pipeline_create(int32_t max_chunks, rota_attn_pipeline** out) {
+  if (!out || max_chunks < 1 || max_chunks > (1 << 16)) return ROTA_ERR_INVALID_ARG;
+  *out = nullptr;
+  auto* pl = new (std::nothrow) rota_attn_pipeline;
+  if (!pl) return ROTA_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&pl->device);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&pl->h2d, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&pl->d2h, cudaStreamNonBlocking);
+  for (int i = 0; e == cudaSuccess && i < 2 * max_chunks + 2; ++i) {
+    cudaEvent_t ev = nullptr;
+    e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+    if (e == cudaSuccess) pl->events.push_back(ev);
+  }
+  if (e != cudaSuccess) {
+    rota_attn_pipeline_destroy(pl);
+    return cuda_status(e);
+  }
+  *out = pl;
+  return ROTA_OK;
+}
+
+rota_status rota_attn_pipeline_destroy(rota_attn_pipeline* pl) {
+  if (!pl) return ROTA_OK;
+  cudaError_t first = cudaSuccess;
+  auto keep = [&](cudaError_t e) { if (first == cudaSuccess) first = e; };
+  for (cudaEvent_t ev : pl->events) keep(cudaEventDestroy(ev));
+  if (pl->h2d) keep(cudaStreamDestroy(pl->h2d));
+  if (pl->d2h) keep(cudaStreamDestroy(pl->d2h));
+  delete pl;
+  return cuda_status(first);
+}
+
+int32_t rota_attn_pipeline_chunk_heads(const rota_attn_desc* d, int32_t num_sms) {
+  if (rota_attn_validate(d) != ROTA_OK) return 0;
+  if (num_sms < 1) num_sms = 148;
+  // INT4 CTAs per head; a chunk of h heads takes ceil(h * cph / num_sms) waves
+  // of the attention kernel.  The copies before the first chunk and after the
+  // last are not hidden: about 1.4 heads of compute per head of chunk (fp16
+  // Q/K/V in and fp32 O out over PCIe against the attention of one head).
+  // Each chunk also pays its own prologue and launches, about 0.05 waves.
+  const long long cph = (d->N + rota::kRowsPerCta - 1) / rota::kRowsPerCta;
+  int32_t best = 1;
+  double best_cost = 1e300;
+  for (int32_t h = 1; h <= d->H; ++h) {
+    double waves = 0.0;
+    for (int32_t h0 = 0; h0 < d->H; h0 += h) {
+      const long long nh = std::min<int32_t>(h, d->H - h0);
+      waves += static_cast<double>((nh * cph + num_sms - 1) / num_sms);
+    }
+    const double chunks = static_cast<double>(d->B) * ((d->H + h - 1) / h);
+    const double cost = d->B * waves + 1.4 * static_cast<double>(h * cph) / num_sms + 0.05 * chunks;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = h;
+    }
+  }
+  return best;
+}
+
+rota_status rota_attn_forward_host(const rota_attn_desc* d, const uint16_t* q_host, const uint16_t* k_host,
+                                   const uint16_t* v_host, const uint8_t* head_flags, float* out_host,
+                                   uint16_t* q_dev, uint16_t* k_dev, uint16_t* v_dev, float* out_dev,
+                                   const rota_attn_buffers* buf, int32_t heads_per_chunk, rota_attn_pipeline* pl,
+                                   void* stream) {
+  rota_status st = rota_attn_validate(d);
+  if (st != ROTA_OK) return st;
+  if (!buf || !pl || !q_host || !k_host || !v_host || !out_host || !q_dev || !k_dev || !v_dev || !out_dev)
+    return ROTA_ERR_INVALID_ARG;
+  if (heads_per_chunk < 0) return ROTA_ERR_INVALID_ARG;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (dev != pl->device) return ROTA_ERR_INVALID_ARG;
+  int nsm = 148;
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int32_t hpc = heads_per_chunk ? std::min(heads_per_chunk, d->H) : rota_attn_pipeline_chunk_heads(d, nsm);
+  const int32_t chunks_per_b = (d->H + hpc - 1) / hpc;
+  const long long nchunks = static_cast<long long>(d->B) * chunks_per_b;
+  if (2 * nchunks + 2 > static_cast<long long>(pl->events.size())) return ROTA_ERR_UNSUPPORTED;
+
+  size_t sz[ROTA_BUF_COUNT];
+  if ((st = rota_attn_buffer_sizes(d, sz)) != ROTA_OK) return st;
+  const size_t heads = static_cast<size_t>(d->B) * d->H;
+  const size_t elems_per_head = static_cast<size_t>(d->N) * d->head_dim;
+  auto shift = [&](auto* ptr, int buf_index, size_t head) {
+    using T = std::remove_pointer_t<decltype(ptr)>;
+    if (!ptr) return ptr;
+    return reinterpret_cast<T*>(reinterpret_cast<std::conditional_t<std::is_const_v<T>, const uint8_t*, uint8_t*>>(ptr) +
+                                sz[buf_index] / heads * head);
+  };
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaEvent_t* ev = pl->events.data();
+  cudaEvent_t ev_start = ev[0], ev_end = ev[1];
+  // everything already on `stream` (an earlier call reading q_dev ... out_dev) comes first
+  if ((e = cudaEventRecord(ev_start, s)) != cudaSuccess) return cuda_status(e);
+  if ((e = cudaStreamWaitEvent(pl->h2d, ev_start, 0)) != cudaSuccess) return cuda_status(e);
+  if ((e = cudaStreamWaitEvent(pl->d2h, ev_start, 0)) != cudaSuccess) return cuda_status(e);
+
+  rota_status result = ROTA_OK;
+  long long c = 0;
+  for (int32_t b = 0; b < d->B && result == ROTA_OK; ++b) {
+    for (int32_t h0 = 0; h0 < d->H && result == ROTA_OK; h0 += hpc, ++c) {
+      const int32_t nh = std::min(hpc, d->H - h0);
+      const size_t head = static_cast<size_t>(b) * d->H + h0;
+      const size_t off = head * elems_per_head, n_in = nh * elems_per_head;
+      cudaEvent_t ev_in = ev[2 + 2 * c], ev_done = ev[3 + 2 * c];
+      // inputs of the chunk
+      e = cudaMemcpyAsync(q_dev + off, q_host + off, n_in * 2, cudaMemcpyHostToDevice, pl->h2d);
+      if (e == cudaSuccess) e = cudaMemcpyAsync(k_dev + off, k_host + off, n_in * 2, cudaMemcpyHostToDevice, pl->h2d);
+      if (e == cudaSuccess) e = cudaMemcpyAsync(v_dev + off, v_host + off, n_in * 2, cudaMemcpyHostToDevice, pl->h2d);
+      if (e == cudaSuccess) e = cudaEventRecord(ev_in, pl->h2d);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_in, 0);
+      if (e != cudaSuccess) { result = cuda_status(e); break; }
+      // the chunk as a problem of its own: one batch entry, nh heads
+      rota_attn_desc cd = *d;
+      cd.B = 1;
+      cd.H = nh;
+      rota_attn_buffers cb = *buf;
+      cb.q_codes = shift(buf->q_codes, ROTA_BUF_Q_CODES, head);
+      cb.k_codes = shift(buf->k_codes, ROTA_BUF_K_CODES, head);
+      cb.q_scale = shift(buf->q_scale, ROTA_BUF_Q_SCALE, head);
+      cb.k_scale = shift(buf->k_scale, ROTA_BUF_K_SCALE, head);
+      cb.v_codes = shift(buf->v_codes, ROTA_BUF_V_CODES, head);
+      cb.v_scale = shift(buf->v_scale, ROTA_BUF_V_SCALE, head);
+      cb.q_rope = shift(buf->q_rope, ROTA_BUF_Q_ROPE, head);
+      cb.k_rope = shift(buf->k_rope, ROTA_BUF_K_ROPE, head);
+      cb.int4_work = shift(buf->int4_work, ROTA_BUF_INT4_WORK, head);
+      const uint8_t* flags = head_flags ? head_flags + h0 : nullptr;
+      result = rota_attn_prepare_qk(&cd, q_dev + off, k_dev + off, v_dev + off, flags, &cb, s);
+      if (result == ROTA_OK) result = rota_attn_fwd_int4(&cd, &cb, flags, out_dev + off, s);
+      if (result == ROTA_OK) result = rota_attn_fwd_fp16_fallback(&cd, &cb, v_dev + off, flags, out_dev + off, s);
+      if (result != ROTA_OK) break;
+      // its output
+      e = cudaEventRecord(ev_done, s);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(pl->d2h, ev_done, 0);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(out_host + off, out_dev + off, n_in * 4, cudaMemcpyDeviceToHost, pl->d2h);
+      if (e != cudaSuccess) result = cuda_status(e);
+    }
+  }
+  // `stream` continues after the last copy-out (also on an error path, so that
+  // both copy streams are joined before the caller reuses the buffers)
+  e = cudaEventRecord(ev_end, pl->d2h);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_end, 0);
+  if (e == cudaSuccess) e = cudaEventRecord(ev_end, pl->h2d);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_end, 0);
+  if (result == ROTA_OK && e != cudaSuccess) result = cuda_status(e);
+  return result;
 }
 
 rota_status rota_attn_get_error(void* stream) {

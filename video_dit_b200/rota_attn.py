@@ -62,6 +62,11 @@ _SIGS = {
     "rota_attn_debug_pcode": ([_P, _P, ctypes.c_int64, _P], ctypes.c_int),
     "rota_attn_debug_inject_timeout": ([ctypes.c_int32, ctypes.c_uint64], ctypes.c_int),
     "rota_attn_fwd_int4_noalloc": ([_D, _P, _P, _P, _P, _P], ctypes.c_int),
+    "rota_attn_pipeline_create": ([ctypes.c_int32, ctypes.POINTER(_P)], ctypes.c_int),
+    "rota_attn_pipeline_destroy": ([_P], ctypes.c_int),
+    "rota_attn_pipeline_chunk_heads": ([_D, ctypes.c_int32], ctypes.c_int32),
+    "rota_attn_forward_host": ([_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _BUF, ctypes.c_int32, _P, _P],
+                               ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -145,6 +150,29 @@ def rota_attn_fwd_int4_noalloc(desc, q, k, v, out, stream=None) -> int:
     device scratch (for callers that cannot allocate device memory)."""
     return _lib.rota_attn_fwd_int4_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                            _stream(stream))
+
+
+def rota_attn_pipeline_create(max_chunks: int):
+    """-> (status, handle): copy streams and events on the current device."""
+    h = _P()
+    st = _lib.rota_attn_pipeline_create(int(max_chunks), ctypes.byref(h))
+    return st, h
+
+
+def rota_attn_pipeline_destroy(handle) -> int:
+    return _lib.rota_attn_pipeline_destroy(handle)
+
+
+def rota_attn_pipeline_chunk_heads(desc, num_sms: int = 0) -> int:
+    return _lib.rota_attn_pipeline_chunk_heads(ctypes.byref(desc), int(num_sms))
+
+
+def rota_attn_forward_host(desc, q_host, k_host, v_host, head_flags, out_host, q_dev, k_dev, v_dev, out_dev,
+                           buffers: rota_attn_buffers, heads_per_chunk: int, pipeline, stream=None) -> int:
+    return _lib.rota_attn_forward_host(ctypes.byref(desc), _ptr(q_host), _ptr(k_host), _ptr(v_host),
+                                       _flags(head_flags), _ptr(out_host), _ptr(q_dev), _ptr(k_dev), _ptr(v_dev),
+                                       _ptr(out_dev), ctypes.byref(buffers), int(heads_per_chunk), pipeline,
+                                       _stream(stream))
 
 
 def rota_attn_get_error(stream=None) -> int:
@@ -234,6 +262,43 @@ class RotaAttention:
         self.prepare(q, k, v, head_flags, stream)
         self.attention(v, head_flags, out, stream)
         return out
+
+    def forward_host(self, q_host, k_host, v_host, head_flags=None, out_host=None, heads_per_chunk: int = 0,
+                     stream=None):
+        """q_host, k_host, v_host: fp16 [B,H,N,d] pinned host tensors -> fp32
+        [B,H,N,d] host tensor, through rota_attn_forward_host (copies of
+        neighbouring head chunks overlap the kernels).  The device staging
+        tensors and the copy pipeline are made on first use and kept.  The
+        result is complete once `stream` (default: the current stream) has
+        reached the end of the call."""
+        import torch
+        if out_host is None:
+            out_host = torch.empty(q_host.shape, dtype=torch.float32, pin_memory=True)
+        d = self.desc
+        if getattr(self, "_stage", None) is None:
+            shape = (d.B, d.H, d.N, d.head_dim)
+            self._stage = tuple(torch.empty(shape, dtype=torch.float16, device=self.device) for _ in range(3)) + (
+                torch.empty(shape, dtype=torch.float32, device=self.device),)
+            st, h = rota_attn_pipeline_create(d.B * d.H)
+            _check(st, "rota_attn_pipeline_create")
+            self._pipeline = h
+        qd, kd, vd, od = self._stage
+        _check(rota_attn_forward_host(d, q_host, k_host, v_host, head_flags, out_host, qd, kd, vd, od, self.buffers,
+                                      heads_per_chunk, self._pipeline, stream), "rota_attn_forward_host")
+        return out_host
+
+    def close(self):
+        """Releases the copy pipeline of forward_host (if one was made)."""
+        h = getattr(self, "_pipeline", None)
+        if h is not None:
+            self._pipeline = None
+            _check(rota_attn_pipeline_destroy(h), "rota_attn_pipeline_destroy")
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
     # views of the intermediate buffers in the documented layouts
     def codes(self):
