@@ -14,7 +14,7 @@
  *   - All tensor pointers are DEVICE pointers allocated by the caller, except
  *     where a parameter is marked "host".  The library never allocates,
  *     never frees and never synchronises (except rota_attn_get_error), apart
- *     from the copy streams and events that rota_attn_pipeline_create makes
+ *     from the streams and events that rota_attn_pipeline_create makes
  *     on request and rota_attn_pipeline_destroy releases.
  *   - fp16 tensors are passed as their uint16_t bit patterns.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream); every
@@ -192,9 +192,11 @@ rota_status rota_attn_fwd_fp16_fallback(const rota_attn_desc* desc, const rota_a
  * The heads of each batch entry are taken in chunks of heads_per_chunk
  * (0 = rota_attn_pipeline_chunk_heads for this device): chunk c's inputs are
  * copied in on the pipeline's host-to-device stream, its prologue, INT4
- * attention and FP16 fallback run on `stream`, and its output is copied out
- * on the device-to-host stream, so the copies of neighbouring chunks overlap
- * chunk c's kernels.  Every result is the one the three calls give on the
+ * attention and FP16 fallback run on `stream` (even c) or on the pipeline's
+ * second compute stream (odd c), and its output is copied out on the
+ * device-to-host stream.  So the copies of neighbouring chunks overlap chunk
+ * c's kernels, and the next chunk's kernels fill the SMs that the last wave of
+ * chunk c's attention leaves idle.  Every result is the one the three calls give on the
  * whole problem (heads are independent).  Ordering: the copies start after
  * the work already enqueued on `stream`, and `stream` continues only after
  * the last copy-out, so out_host is complete once `stream` has reached that
@@ -206,16 +208,18 @@ rota_status rota_attn_fwd_fp16_fallback(const rota_attn_desc* desc, const rota_a
  */
 typedef struct rota_attn_pipeline rota_attn_pipeline;
 
-/* Creates, on the current device, the two copy streams (non-blocking) and the
- * events for up to max_chunks chunks per call.  *out receives the handle. */
+/* Creates, on the current device, the two copy streams and the second compute
+ * stream (all non-blocking) and the events for up to max_chunks chunks per
+ * call.  *out receives the handle. */
 rota_status rota_attn_pipeline_create(int32_t max_chunks, rota_attn_pipeline** out);
 
 /* Releases what rota_attn_pipeline_create made (NULL is a no-op). */
 rota_status rota_attn_pipeline_destroy(rota_attn_pipeline* pipeline);
 
-/* The default chunk size: heads per chunk that minimise the waves of the
- * attention kernel over all chunks plus the unhidden copies of the first and
- * last chunk, for a device with num_sms SMs (0 on an invalid descriptor). */
+/* The default chunk size for a device with num_sms SMs (0 on an invalid
+ * descriptor): the heads per chunk that minimise the unhidden copies of the
+ * first and last chunk plus a fixed cost per chunk (its prologue, widening and
+ * launches), both counted in waves of the attention kernel. */
 int32_t rota_attn_pipeline_chunk_heads(const rota_attn_desc* desc, int32_t num_sms);
 
 rota_status rota_attn_forward_host(const rota_attn_desc* desc, const uint16_t* q_host, const uint16_t* k_host,

@@ -423,6 +423,7 @@ rota_status rota_attn_fwd_fp16_fallback(const rota_attn_desc* d, const rota_attn
 struct rota_attn_pipeline {
   int device = 0;
   cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaStream_t comp2 = nullptr;       // odd chunks compute here, even ones on the caller's stream
   std::vector<cudaEvent_t> events;   // 2 per chunk + 2
 };
 
@@ -434,6 +435,7 @@ rota_status rota_attn_pipeline_create(int32_t max_chunks, rota_attn_pipeline** o
   cudaError_t e = cudaGetDevice(&pl->device);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&pl->h2d, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&pl->d2h, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&pl->comp2, cudaStreamNonBlocking);
   for (int i = 0; e == cudaSuccess && i < 2 * max_chunks + 2; ++i) {
     cudaEvent_t ev = nullptr;
     e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
@@ -454,6 +456,7 @@ rota_status rota_attn_pipeline_destroy(rota_attn_pipeline* pl) {
   for (cudaEvent_t ev : pl->events) keep(cudaEventDestroy(ev));
   if (pl->h2d) keep(cudaStreamDestroy(pl->h2d));
   if (pl->d2h) keep(cudaStreamDestroy(pl->d2h));
+  if (pl->comp2) keep(cudaStreamDestroy(pl->comp2));
   delete pl;
   return cuda_status(first);
 }
@@ -461,22 +464,19 @@ rota_status rota_attn_pipeline_destroy(rota_attn_pipeline* pl) {
 int32_t rota_attn_pipeline_chunk_heads(const rota_attn_desc* d, int32_t num_sms) {
   if (rota_attn_validate(d) != ROTA_OK) return 0;
   if (num_sms < 1) num_sms = 148;
-  // INT4 CTAs per head; a chunk of h heads takes ceil(h * cph / num_sms) waves
-  // of the attention kernel.  The copies before the first chunk and after the
-  // last are not hidden: about 1.4 heads of compute per head of chunk (fp16
-  // Q/K/V in and fp32 O out over PCIe against the attention of one head).
-  // Each chunk also pays its own prologue and launches, about 0.05 waves.
-  const long long cph = (d->N + rota::kRowsPerCta - 1) / rota::kRowsPerCta;
+  // Consecutive chunks compute on two streams, so the attention waves of all
+  // chunks pack about as tightly as one call on the whole problem and the
+  // chunk size does not change them.  What it changes: the copies before the
+  // first chunk and after the last are not hidden (about 1.4 heads of
+  // attention per head of chunk: fp16 Q/K/V in and fp32 O out over PCIe
+  // against one head's attention, in waves of cph / num_sms), and every chunk
+  // pays its own prologue, widening and launches (about 0.05 waves).
+  const double cph = static_cast<double>((d->N + rota::kRowsPerCta - 1) / rota::kRowsPerCta);
   int32_t best = 1;
   double best_cost = 1e300;
   for (int32_t h = 1; h <= d->H; ++h) {
-    double waves = 0.0;
-    for (int32_t h0 = 0; h0 < d->H; h0 += h) {
-      const long long nh = std::min<int32_t>(h, d->H - h0);
-      waves += static_cast<double>((nh * cph + num_sms - 1) / num_sms);
-    }
     const double chunks = static_cast<double>(d->B) * ((d->H + h - 1) / h);
-    const double cost = d->B * waves + 1.4 * static_cast<double>(h * cph) / num_sms + 0.05 * chunks;
+    const double cost = 1.4 * h * cph / num_sms + 0.05 * chunks;
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best = h;
@@ -524,6 +524,7 @@ rota_status rota_attn_forward_host(const rota_attn_desc* d, const uint16_t* q_ho
   if ((e = cudaEventRecord(ev_start, s)) != cudaSuccess) return cuda_status(e);
   if ((e = cudaStreamWaitEvent(pl->h2d, ev_start, 0)) != cudaSuccess) return cuda_status(e);
   if ((e = cudaStreamWaitEvent(pl->d2h, ev_start, 0)) != cudaSuccess) return cuda_status(e);
+  if ((e = cudaStreamWaitEvent(pl->comp2, ev_start, 0)) != cudaSuccess) return cuda_status(e);
 
   rota_status result = ROTA_OK;
   long long c = 0;
@@ -533,12 +534,15 @@ rota_status rota_attn_forward_host(const rota_attn_desc* d, const uint16_t* q_ho
       const size_t head = static_cast<size_t>(b) * d->H + h0;
       const size_t off = head * elems_per_head, n_in = nh * elems_per_head;
       cudaEvent_t ev_in = ev[2 + 2 * c], ev_done = ev[3 + 2 * c];
+      // consecutive chunks compute on two streams, so that the next chunk's
+      // kernels fill the SMs the last wave of this chunk's attention leaves idle
+      cudaStream_t cs = (c & 1) ? pl->comp2 : s;
       // inputs of the chunk
       e = cudaMemcpyAsync(q_dev + off, q_host + off, n_in * 2, cudaMemcpyHostToDevice, pl->h2d);
       if (e == cudaSuccess) e = cudaMemcpyAsync(k_dev + off, k_host + off, n_in * 2, cudaMemcpyHostToDevice, pl->h2d);
       if (e == cudaSuccess) e = cudaMemcpyAsync(v_dev + off, v_host + off, n_in * 2, cudaMemcpyHostToDevice, pl->h2d);
       if (e == cudaSuccess) e = cudaEventRecord(ev_in, pl->h2d);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_in, 0);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, ev_in, 0);
       if (e != cudaSuccess) { result = cuda_status(e); break; }
       // the chunk as a problem of its own: one batch entry, nh heads
       rota_attn_desc cd = *d;
@@ -555,12 +559,12 @@ rota_status rota_attn_forward_host(const rota_attn_desc* d, const uint16_t* q_ho
       cb.k_rope = shift(buf->k_rope, ROTA_BUF_K_ROPE, head);
       cb.int4_work = shift(buf->int4_work, ROTA_BUF_INT4_WORK, head);
       const uint8_t* flags = head_flags ? head_flags + h0 : nullptr;
-      result = rota_attn_prepare_qk(&cd, q_dev + off, k_dev + off, v_dev + off, flags, &cb, s);
-      if (result == ROTA_OK) result = rota_attn_fwd_int4(&cd, &cb, flags, out_dev + off, s);
-      if (result == ROTA_OK) result = rota_attn_fwd_fp16_fallback(&cd, &cb, v_dev + off, flags, out_dev + off, s);
+      result = rota_attn_prepare_qk(&cd, q_dev + off, k_dev + off, v_dev + off, flags, &cb, cs);
+      if (result == ROTA_OK) result = rota_attn_fwd_int4(&cd, &cb, flags, out_dev + off, cs);
+      if (result == ROTA_OK) result = rota_attn_fwd_fp16_fallback(&cd, &cb, v_dev + off, flags, out_dev + off, cs);
       if (result != ROTA_OK) break;
       // its output
-      e = cudaEventRecord(ev_done, s);
+      e = cudaEventRecord(ev_done, cs);
       if (e == cudaSuccess) e = cudaStreamWaitEvent(pl->d2h, ev_done, 0);
       if (e == cudaSuccess)
         e = cudaMemcpyAsync(out_host + off, out_dev + off, n_in * 4, cudaMemcpyDeviceToHost, pl->d2h);
@@ -572,6 +576,8 @@ rota_status rota_attn_forward_host(const rota_attn_desc* d, const uint16_t* q_ho
   e = cudaEventRecord(ev_end, pl->d2h);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_end, 0);
   if (e == cudaSuccess) e = cudaEventRecord(ev_end, pl->h2d);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_end, 0);
+  if (e == cudaSuccess) e = cudaEventRecord(ev_end, pl->comp2);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_end, 0);
   if (result == ROTA_OK && e != cudaSuccess) result = cuda_status(e);
   return result;
