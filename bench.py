@@ -135,7 +135,7 @@ def workload_config(w, l2_note):
 # current kernels on the F = 3 sweep point (B=1, H=40, N=4680, profiles/), per
 # (head, token): the traffic is the K/V images or tiles and the output, linear
 # in B * heads * N.  None = no capture of the current kernel version.
-TRAFFIC_PER_HEAD_TOKEN = {"attn_int4_kernel": 1034.97, "attn_fp16_kernel": 1080.38}
+TRAFFIC_PER_HEAD_TOKEN = {"attn_int4_kernel": 1035.70, "attn_fp16_kernel": 1076.75}
 
 
 def traffic_per_launch(kernel, w, heads):
@@ -207,6 +207,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=128)      # per step of --impl reference
     ap.add_argument("--cpu-rows", type=int, default=1024)     # the cpu_baseline sample (about 10 s)
     ap.add_argument("--chunk-heads", type=int, default=0)     # heads per chunk of the e2e pipeline (0: library default)
+    ap.add_argument("--no-e2e", action="store_true")          # skip the end-to-end loop (profiling runs)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -288,24 +289,27 @@ def main():
     t_int4 = [e[1].elapsed_time(e[2]) for e in evs]
     t_f16 = [e[2].elapsed_time(e[3]) for e in evs]
 
-    # end to end through the public API: pinned host inputs in, fp32 output back, every step
-    # (rota_attn_forward_host: head chunks, copies of neighbouring chunks overlapping the kernels)
-    e2e_steps = max(3, min(args.steps, 10))
-    chunk_heads = args.chunk_heads or ra.rota_attn_pipeline_chunk_heads(
-        att.desc, torch.cuda.get_device_properties(dev).multi_processor_count)
-    att.forward_host(qh, kh, vh, flags, out_h, heads_per_chunk=chunk_heads, stream=stream)   # staging, warm-up
-    barrier()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        att.forward_host(qh, kh, vh, flags, out_h, heads_per_chunk=chunk_heads, stream=stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
+    ms_e2e, chunk_heads = 0.0, None
+    if not args.no_e2e:
+        # end to end through the public API: pinned host inputs in, fp32 output back, every step
+        # (rota_attn_forward_host: head chunks, copies of neighbouring chunks overlapping the kernels)
+        e2e_steps = max(3, min(args.steps, 10))
+        chunk_heads = args.chunk_heads or ra.rota_attn_pipeline_chunk_heads(
+            att.desc, torch.cuda.get_device_properties(dev).multi_processor_count)
+        att.forward_host(qh, kh, vh, flags, out_h, heads_per_chunk=chunk_heads, stream=stream)   # staging, warm-up
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            att.forward_host(qh, kh, vh, flags, out_h, heads_per_chunk=chunk_heads, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
     clocks = sampler.stop()
-    ms_e2e = e0.elapsed_time(e1) / e2e_steps
+    if not args.no_e2e:
+        ms_e2e = e0.elapsed_time(e1) / e2e_steps
     st = ra.rota_attn_get_error()
     if st != ra.ROTA_OK:
         raise RuntimeError(f"device error in the timed region: {ra.rota_attn_status_string(st)}")
@@ -359,9 +363,10 @@ def main():
             "breakdown_ms": {"prologue": ms_pro, "int4_attention": ms_int4, "fp16_fallback": ms_f16},
             "prologue_gbs": pro_bytes / (ms_pro * 1e-3) / 1e9,
             "roofline": rl,
-            "e2e": {"value": ops * world / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
-                    "heads_per_chunk": chunk_heads},
+            "e2e": None if args.no_e2e else {
+                "value": ops * world / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+                "heads_per_chunk": chunk_heads},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }
