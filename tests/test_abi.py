@@ -106,3 +106,50 @@ def test_kappa_matches_oracle_definition(ra):
     for d in (64, 128):
         sm = np.float32(1 / np.sqrt(d))
         assert ra.kappa(d) == np.float32(np.float64(sm) * 1.4426950408889634074)
+
+
+# ----------------------------------------------- host-to-host pipeline (host logic)
+
+@pytest.mark.parametrize("name", ["wan480", "wan720", "hunyuan"])
+def test_chunk_heads_default_is_one_head_on_large_problems(ra, name):
+    # one head's fp16 Q/K/V in and fp32 O out cost more than a chunk's fixed
+    # overhead on these sizes, so the unhidden first and last copies decide
+    assert ra.rota_attn_pipeline_chunk_heads(_desc(ra, synth.WORKLOADS[name]), 148) == 1
+
+
+def test_chunk_heads_grows_when_heads_are_small(ra):
+    # N = 256: a head is 1 attention CTA, so the per-chunk cost dominates
+    w = synth.scaled(synth.WORKLOADS["wan480"], "small", H=40, grid=(1, 4, 64))
+    h = ra.rota_attn_pipeline_chunk_heads(_desc(ra, w), 148)
+    assert 1 < h <= 40
+    # a larger N never asks for more heads per chunk
+    prev = h
+    for grid in [(1, 16, 64), (1, 64, 64), (4, 64, 64)]:
+        cur = ra.rota_attn_pipeline_chunk_heads(_desc(ra, synth.scaled(w, "g", grid=grid)), 148)
+        assert 1 <= cur <= prev
+        prev = cur
+
+
+def test_chunk_heads_invalid_descriptor(ra):
+    d = _desc(ra, synth.WORKLOADS["wan480"])
+    d.head_dim = 96
+    assert ra.rota_attn_pipeline_chunk_heads(d, 148) == 0
+    # num_sms <= 0 falls back to the B200's 148
+    d = _desc(ra, synth.WORKLOADS["wan480"])
+    assert ra.rota_attn_pipeline_chunk_heads(d, 0) == ra.rota_attn_pipeline_chunk_heads(d, 148)
+
+
+def test_pipeline_arguments_rejected_before_any_cuda_call(ra):
+    h = ctypes.c_void_p()
+    assert ra._lib.rota_attn_pipeline_create(0, ctypes.byref(h)) == ra.ROTA_ERR_INVALID_ARG
+    assert ra._lib.rota_attn_pipeline_create(4, None) == ra.ROTA_ERR_INVALID_ARG
+    assert ra.rota_attn_pipeline_destroy(None) == ra.ROTA_OK
+    d = _desc(ra, synth.WORKLOADS["tiny"])
+    b = ra.rota_attn_buffers()
+    nul = [None] * 4
+    # null host / device pointers and a null pipeline
+    assert ra._lib.rota_attn_forward_host(ctypes.byref(d), None, None, None, None, None, *nul, ctypes.byref(b), 0,
+                                          None, None) == ra.ROTA_ERR_INVALID_ARG
+    d.head_dim = 96
+    assert ra._lib.rota_attn_forward_host(ctypes.byref(d), None, None, None, None, None, *nul, ctypes.byref(b), 0,
+                                          None, None) == ra.ROTA_ERR_INVALID_ARG

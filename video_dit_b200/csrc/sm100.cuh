@@ -54,21 +54,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// try_wait with a suspend-time hint: the thread sleeps (issuing nothing) until
-// the phase completes or about `hint_ns` pass, so waiting warps leave the
-// issue slots of their SM sub-partition to the warps that compute.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait for phase `parity` of `bar` to complete, for at most `limit_ns`.
 // Returns false (and records kDevTimeout) if the limit ran out.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
@@ -134,11 +119,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, 
       : "memory");
 }
 
-// Generic-proxy writes to shared memory -> visible to the async proxy (MMA).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // --------------------------------------------------------------- tcgen05 ---
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -197,45 +177,12 @@ __host__ __device__ constexpr uint32_t idesc(uint32_t dfmt, uint32_t afmt, uint3
          ((M >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(id), "r"(acc)
-      : "memory");
-}
-
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(id), "r"(acc)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(id), "r"(acc)
-      : "memory");
-}
-
-// Same MMAs with the descriptors given as (lo, hi) 32-bit halves, so a caller
-// can keep the constant high words in registers and step the start address
-// with one add; `acc` selects accumulate (1) or overwrite (0) at compile time.
-template <int ACC>
-__device__ __forceinline__ void mma_f8f6f4_lh(uint32_t d_tmem, uint32_t alo, uint32_t ahi, uint32_t blo, uint32_t bhi,
-                                              uint32_t id) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 a, b;\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "mov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %4};\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %6, p;\n\t}" ::"r"(d_tmem),
-      "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "n"(ACC), "r"(id)
       : "memory");
 }
 
@@ -249,20 +196,6 @@ __device__ __forceinline__ void mma_f8f6f4_ts(uint32_t d_tmem, uint32_t a_tmem, 
       "mov.b64 b, {%2, %3};\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], b, %5, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "r"(blo), "r"(bhi), "n"(ACC), "r"(id)
-      : "memory");
-}
-
-// The same for kind::f16 (both operands f16, or both bf16, as the
-// instruction descriptor says).
-template <int ACC>
-__device__ __forceinline__ void mma_f16_lh(uint32_t d_tmem, uint32_t alo, uint32_t ahi, uint32_t blo, uint32_t bhi,
-                                           uint32_t id) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 a, b;\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "mov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %4};\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %6, p;\n\t}" ::"r"(d_tmem),
-      "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "n"(ACC), "r"(id)
       : "memory");
 }
 
@@ -305,17 +238,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
         "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
         "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-}
-
-// 32 lanes x 16 consecutive 32-bit columns.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
       : "memory");
 }
@@ -389,14 +311,6 @@ __device__ __forceinline__ void tmem_wait_dep2(uint32_t (&a)[32], uint32_t (&b)[
                "+r"(b[24]), "+r"(b[25]), "+r"(b[26]), "+r"(b[27]), "+r"(b[28]), "+r"(b[29]), "+r"(b[30]), "+r"(b[31])
                :: "memory");
 }
-__device__ __forceinline__ void tmem_wait_dep16(uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.wait::ld.sync.aligned;"
-      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
-      :
-      : "memory");
-}
 __device__ __forceinline__ void tmem_wait_dep1(uint32_t& r) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r) : : "memory");
 }
@@ -419,11 +333,6 @@ __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, f
 }
 __device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
   const float2 r = __fadd2_rn(make_float2(a0, a1), make_float2(b0, b1));
-  d0 = r.x;
-  d1 = r.y;
-}
-__device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  const float2 r = __fmul2_rn(make_float2(a0, a1), make_float2(b0, b1));
   d0 = r.x;
   d1 = r.y;
 }
