@@ -238,6 +238,29 @@ def test_pcode_dense_sample_matches_threshold_form():
     assert np.array_equal(u.astype(np.int64), want)
 
 
+def _max_key_codes(lo: float, hi: float, n: int = 20000, seed: int = 12):
+    """P code of the key that sets the running max, m = RN(S c), for n random
+    (S_int, c) with |S c| in [lo, hi): d = RN(S c - m) (the one rounding of the
+    fma; S c - m is exact in double)."""
+    rng = np.random.default_rng(seed)
+    s_int = rng.integers(1, 49 * 128, n).astype(np.float64)
+    x = np.exp(rng.uniform(np.log(lo), np.log(hi), n))
+    c = (x / s_int).astype(np.float32).astype(np.float64)
+    m = (s_int * c).astype(np.float32).astype(np.float64)
+    d = (s_int * c - m).astype(np.float32)
+    return oracle.pcode_array(d)
+
+
+def test_max_key_keeps_code_15_below_2_pow_20():
+    """The row sum is at least 15 (the key that sets the max has code 15) while
+    the logits stay below 2^20: there the rounding of m moves that key's
+    exponent by at most half an ulp of m, <= 2^-5, well inside log2(14.5/15).
+    Beyond 2^21 the half ulp exceeds it and the code can drop."""
+    assert (_max_key_codes(1e-3, 2.0 ** 20) == 15).all()
+    assert math.log2(14.5 / 15) < -(2.0 ** -5)
+    assert (_max_key_codes(2.0 ** 21, 2.0 ** 24) < 15).any()
+
+
 # ------------------------------------------------------ whole pipeline ---
 
 def _tiny(**kw):

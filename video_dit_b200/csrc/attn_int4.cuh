@@ -18,8 +18,10 @@
 // parts of 8 significant bits each, s_hi = s with its low 16 mantissa bits
 // cleared and s_lo = (s - s_hi) likewise (s - s_hi - s_lo < 2^-14 s); a code
 // (3 bits of magnitude) times either part has at most 11 significant bits, so
-// the V' tiles v * s_hi and v * s_lo are exact fp16 values (within fp16's
-// range), and the P codes u in 0..15 are exact fp16 too.  tcgen05.mma
+// the V' tiles v * s_hi and v * s_lo are exact fp16 values while they are
+// normal fp16 numbers (|v * s_hi| <= 7 s <= the block's max |V|, so never
+// above the fp16 range; a very small scale makes v * s_lo subnormal, rounded
+// to within 2^-25 absolute), and the P codes u in 0..15 are exact fp16 too.  tcgen05.mma
 // kind::f16 then forms s_hi * sum_k u v and s_lo * sum_k u v exactly (each
 // block sum is an integer below 2^13 times one part: at most 21 significant
 // bits) and adds them to O in TMEM.  So O accumulates on the tensor core
