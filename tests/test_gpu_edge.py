@@ -4,7 +4,8 @@ so c = 0 for that block), V near the fp16 maximum with logits up to the
 method's 2^20 range, and V small
 enough that the low part of the V' split (v * s_lo) is an fp16 subnormal.
 Codes and scales byte-exact, S and P codes bit-exact, outputs within the
-parity tolerance of the oracle's double result."""
+parity tolerance of the oracle's double result (scaled with |O| beyond the
+workloads' output range)."""
 import numpy as np
 import pytest
 
@@ -76,7 +77,11 @@ def test_edge_case_parity(case):
         o = o_ref if hh == h else oracle.attn_int4(ref, w.N, sm_scale(w), 0, hh, 0, w.N)
         assert np.isfinite(out[0, hh]).all(), hh
         e, rel, cos = row_stats(out[0, hh], o)
-        assert e <= TOL, (hh, e, rel, cos)
+        # the 2e-3 bar is for outputs up to ~32 (the workloads' range with x8 V
+        # outlier tokens); fp32 accumulation and the < 2^-14 residual of the V
+        # scale split are relative errors, so beyond that the bar scales with |O|
+        tol = TOL * max(1.0, float(np.abs(o).max()) / 32.0)
+        assert e <= tol, (hh, e, tol, rel, cos)
     if case == "zeros":
         assert not out.any()                       # every code 0: O = 0 exactly
     if case == "one_token":
