@@ -228,6 +228,38 @@ rota_status rota_attn_forward_host(const rota_attn_desc* desc, const uint16_t* q
                                    const rota_attn_buffers* buf, int32_t heads_per_chunk,
                                    rota_attn_pipeline* pipeline, void* stream);
 
+/*
+ * Choosing the FP16-fallback heads.  The paper keeps accuracy-sensitive
+ * attention blocks and denoising steps in FP16 but gives no rule for which
+ * ones; these two calls measure it on a calibration call and turn the result
+ * into the host flag array the attention calls take.
+ *
+ * rota_attn_head_error: out_test, out_ref: device fp32 [B,H,N,head_dim]
+ * (16-byte aligned), typically the output with every head on the INT4 path
+ * and the output with every head on the FP16 fallback for the same inputs.
+ * sums: device double [B*H*2] (8-byte aligned), overwritten with, per
+ * (b, h), sum (out_test - out_ref)^2 and sum out_ref^2 (fp64 accumulation;
+ * the summation order varies between runs, so the last bits may too).
+ * Enqueued on `stream` (a memset and one kernel); no synchronisation.
+ */
+rota_status rota_attn_head_error(const rota_attn_desc* desc, const float* out_test, const float* out_ref,
+                                 double* sums, void* stream);
+
+/*
+ * Host only.  sums: host double [B*H*2] as rota_attn_head_error writes them.
+ * A head's error is the largest relative Frobenius error over the batch,
+ * sqrt(sum diff^2 / sum ref^2) (infinite for NaN sums, or for a zero
+ * reference with a non-zero difference; 0 when both are zero).  Heads whose
+ * error exceeds max_rel_err are flagged, the largest errors first, at most
+ * max_fp16_heads of them (< 0: no limit; ties go to the lower head index).
+ * flags: host uint8 [H] (1 = FP16 fallback), overwritten; rel_err: host
+ * float [H] receiving the errors, or NULL.  ROTA_ERR_INVALID_ARG for null
+ * sums / flags, B < 1, H outside [1, 256] or a negative / non-finite
+ * max_rel_err.
+ */
+rota_status rota_attn_select_fp16_heads(const double* sums, int32_t B, int32_t H, float max_rel_err,
+                                        int32_t max_fp16_heads, float* rel_err, uint8_t* flags);
+
 /* Synchronises `stream`, then returns and clears the device error word
  * (ROTA_OK, ROTA_ERR_TIMEOUT or ROTA_ERR_DEVICE), or ROTA_ERR_CUDA if the
  * synchronisation itself failed. */

@@ -153,3 +153,62 @@ def test_pipeline_arguments_rejected_before_any_cuda_call(ra):
     d.head_dim = 96
     assert ra._lib.rota_attn_forward_host(ctypes.byref(d), None, None, None, None, None, *nul, ctypes.byref(b), 0,
                                           None, None) == ra.ROTA_ERR_INVALID_ARG
+
+
+# ----------------------------------------------- FP16-head selection (host rule)
+
+def _sums(rel, ref=1.0):
+    """Per-head sums (diff^2, ref^2) giving relative errors `rel` (B rows)."""
+    rel = np.atleast_2d(np.asarray(rel, np.float64))
+    out = np.zeros(rel.shape + (2,), np.float64)
+    out[..., 0] = (rel * ref) ** 2
+    out[..., 1] = ref ** 2
+    return out.reshape(-1)
+
+
+def test_select_threshold_and_order(ra):
+    st, flags, rel = ra.rota_attn_select_fp16_heads(_sums([0.01, 0.2, 0.05, 0.3, 0.11]), 1, 5, 0.1)
+    assert st == ra.ROTA_OK
+    assert flags.tolist() == [0, 1, 0, 1, 1]
+    assert np.allclose(rel, [0.01, 0.2, 0.05, 0.3, 0.11], rtol=1e-6)
+    # a budget keeps the worst ones
+    _, flags, _ = ra.rota_attn_select_fp16_heads(_sums([0.01, 0.2, 0.05, 0.3, 0.11]), 1, 5, 0.1, 2)
+    assert flags.tolist() == [0, 1, 0, 1, 0]
+    _, flags, _ = ra.rota_attn_select_fp16_heads(_sums([0.01, 0.2, 0.05, 0.3, 0.11]), 1, 5, 0.1, 0)
+    assert not flags.any()
+    # nothing above the threshold
+    _, flags, _ = ra.rota_attn_select_fp16_heads(_sums([0.01, 0.02]), 1, 2, 0.5)
+    assert not flags.any()
+
+
+def test_select_worst_batch_entry_and_ties(ra):
+    # B = 2: head 0 is fine in entry 0 but bad in entry 1
+    s = _sums([[0.01, 0.2, 0.2], [0.4, 0.01, 0.2]])
+    _, flags, rel = ra.rota_attn_select_fp16_heads(s, 2, 3, 0.1, 2)
+    assert np.allclose(rel, [0.4, 0.2, 0.2], rtol=1e-6)
+    assert flags.tolist() == [1, 1, 0]            # tie between heads 1 and 2: the lower index
+
+
+def test_select_degenerate_sums(ra):
+    s = _sums([0.0, 0.0, 0.0, 0.0])
+    s[2 * 1] = np.nan                             # NaN difference: infinite error
+    s[2 * 2 + 1] = 0.0                            # zero reference, zero difference: error 0
+    s[2 * 3], s[2 * 3 + 1] = 1.0, 0.0             # zero reference, non-zero difference: infinite
+    _, flags, rel = ra.rota_attn_select_fp16_heads(s, 1, 4, 0.1)
+    assert flags.tolist() == [0, 1, 0, 1]
+    assert np.isinf(rel[1]) and np.isinf(rel[3]) and rel[2] == 0.0
+
+
+@pytest.mark.parametrize("B,H,thr", [(0, 4, 0.1), (1, 0, 0.1), (1, 257, 0.1), (1, 4, -1.0), (1, 4, float("nan"))])
+def test_select_rejects(ra, B, H, thr):
+    s = np.zeros(max(1, B) * max(1, H) * 2)
+    flags = np.zeros(max(1, H), np.uint8)
+    st = ra._lib.rota_attn_select_fp16_heads(s.ctypes.data, B, H, thr, -1, None, flags.ctypes.data)
+    assert st == ra.ROTA_ERR_INVALID_ARG
+
+
+def test_select_rejects_null_pointers(ra):
+    s = np.zeros(8)
+    flags = np.zeros(4, np.uint8)
+    assert ra._lib.rota_attn_select_fp16_heads(None, 1, 4, 0.1, -1, None, flags.ctypes.data) == ra.ROTA_ERR_INVALID_ARG
+    assert ra._lib.rota_attn_select_fp16_heads(s.ctypes.data, 1, 4, 0.1, -1, None, None) == ra.ROTA_ERR_INVALID_ARG

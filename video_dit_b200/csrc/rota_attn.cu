@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <limits>
 #include <mutex>
 #include <new>
 #include <type_traits>
@@ -15,6 +16,7 @@
 
 #include "../../include/rota_attn.h"
 #include "attn_fp16.cuh"
+#include "calib.cuh"
 #include "attn_int4.cuh"
 #include "prologue.cuh"
 
@@ -581,6 +583,58 @@ rota_status rota_attn_forward_host(const rota_attn_desc* d, const uint16_t* q_ho
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_end, 0);
   if (result == ROTA_OK && e != cudaSuccess) result = cuda_status(e);
   return result;
+}
+
+// ---------------------------------------------------------------------------
+// Choosing the FP16-fallback heads from a calibration call.
+// ---------------------------------------------------------------------------
+rota_status rota_attn_head_error(const rota_attn_desc* d, const float* out_test, const float* out_ref,
+                                 double* sums, void* stream) {
+  rota_status st = rota_attn_validate(d);
+  if (st != ROTA_OK) return st;
+  if (!out_test || !out_ref || !sums || !aligned16(out_test) || !aligned16(out_ref) ||
+      (reinterpret_cast<uintptr_t>(sums) & 7u))
+    return ROTA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint64_t heads = static_cast<uint64_t>(d->B) * d->H;
+  const uint64_t n4 = static_cast<uint64_t>(d->N) * d->head_dim / 4;
+  cudaError_t e = cudaMemsetAsync(sums, 0, heads * 2 * sizeof(double), s);
+  if (e != cudaSuccess) return cuda_status(e);
+  const uint64_t slices = std::min<uint64_t>(64, (n4 + 8 * rota::kCalibThreads - 1) / (8 * rota::kCalibThreads));
+  const dim3 grid(static_cast<unsigned>(heads), static_cast<unsigned>(std::max<uint64_t>(1, slices)));
+  rota::head_error_kernel<<<grid, rota::kCalibThreads, 0, s>>>(out_test, out_ref, n4, sums);
+  return cuda_status(cudaGetLastError());
+}
+
+rota_status rota_attn_select_fp16_heads(const double* sums, int32_t B, int32_t H, float max_rel_err,
+                                        int32_t max_fp16_heads, float* rel_err, uint8_t* flags) {
+  if (!sums || !flags || B < 1 || H < 1 || H > 256 || !(max_rel_err >= 0.f) || !std::isfinite(max_rel_err))
+    return ROTA_ERR_INVALID_ARG;
+  // per head: the worst batch entry's relative Frobenius error
+  float rel[256];
+  for (int32_t h = 0; h < H; ++h) {
+    double worst = 0.0;
+    for (int32_t b = 0; b < B; ++b) {
+      const double e = sums[2 * (static_cast<size_t>(b) * H + h)];
+      const double q = sums[2 * (static_cast<size_t>(b) * H + h) + 1];
+      double r;
+      if (std::isnan(e) || std::isnan(q)) r = std::numeric_limits<double>::infinity();
+      else if (q > 0.0) r = std::sqrt(e / q);
+      else r = e > 0.0 ? std::numeric_limits<double>::infinity() : 0.0;
+      worst = std::max(worst, r);
+    }
+    rel[h] = static_cast<float>(worst);
+    if (rel_err) rel_err[h] = rel[h];
+    flags[h] = 0;
+  }
+  // candidates above the threshold, worst first (lower head index on ties)
+  int32_t order[256], n = 0;
+  for (int32_t h = 0; h < H; ++h)
+    if (rel[h] > max_rel_err) order[n++] = h;
+  std::stable_sort(order, order + n, [&](int32_t a, int32_t b) { return rel[a] > rel[b]; });
+  const int32_t take = max_fp16_heads < 0 ? n : std::min(n, max_fp16_heads);
+  for (int32_t i = 0; i < take; ++i) flags[order[i]] = 1;
+  return ROTA_OK;
 }
 
 rota_status rota_attn_get_error(void* stream) {

@@ -67,6 +67,9 @@ _SIGS = {
     "rota_attn_pipeline_chunk_heads": ([_D, ctypes.c_int32], ctypes.c_int32),
     "rota_attn_forward_host": ([_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _BUF, ctypes.c_int32, _P, _P],
                                ctypes.c_int),
+    "rota_attn_head_error": ([_D, _P, _P, _P, _P], ctypes.c_int),
+    "rota_attn_select_fp16_heads": ([_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_float, ctypes.c_int32, _P, _P],
+                                    ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -173,6 +176,21 @@ def rota_attn_forward_host(desc, q_host, k_host, v_host, head_flags, out_host, q
                                        _flags(head_flags), _ptr(out_host), _ptr(q_dev), _ptr(k_dev), _ptr(v_dev),
                                        _ptr(out_dev), ctypes.byref(buffers), int(heads_per_chunk), pipeline,
                                        _stream(stream))
+
+
+def rota_attn_head_error(desc, out_test, out_ref, sums, stream=None) -> int:
+    return _lib.rota_attn_head_error(ctypes.byref(desc), _ptr(out_test), _ptr(out_ref), _ptr(sums),
+                                     _stream(stream))
+
+
+def rota_attn_select_fp16_heads(sums: np.ndarray, B: int, H: int, max_rel_err: float, max_fp16_heads: int = -1):
+    """-> (status, flags uint8 [H], rel_err float32 [H]) from host sums [B*H*2]."""
+    sums = np.ascontiguousarray(sums, dtype=np.float64)
+    flags = np.zeros(H, np.uint8)
+    rel = np.zeros(H, np.float32)
+    st = _lib.rota_attn_select_fp16_heads(sums.ctypes.data, int(B), int(H), float(max_rel_err),
+                                          int(max_fp16_heads), rel.ctypes.data, flags.ctypes.data)
+    return st, flags, rel
 
 
 def rota_attn_get_error(stream=None) -> int:
@@ -286,6 +304,28 @@ class RotaAttention:
         _check(rota_attn_forward_host(d, q_host, k_host, v_host, head_flags, out_host, qd, kd, vd, od, self.buffers,
                                       heads_per_chunk, self._pipeline, stream), "rota_attn_forward_host")
         return out_host
+
+    def calibrate_flags(self, q, k, v, max_rel_err: float = 0.1, max_fp16_heads: int = -1, stream=None):
+        """Runs the call twice on these inputs -- every head INT4, then every
+        head on the FP16 fallback -- and flags the heads whose INT4 output is
+        furthest from the FP16 one (rota_attn_head_error +
+        rota_attn_select_fp16_heads).  Returns (flags uint8 [H], relative
+        error float32 [H]).  Needs the FP16 buffers (need_fp16=True)."""
+        import torch
+        if self.q_rope is None:
+            raise ValueError("calibrate_flags needs a RotaAttention made with need_fp16=True")
+        d = self.desc
+        shape = (d.B, d.H, d.N, d.head_dim)
+        o4 = torch.empty(shape, dtype=torch.float32, device=self.device)
+        o16 = torch.empty(shape, dtype=torch.float32, device=self.device)
+        self.forward(q, k, v, np.zeros(d.H, np.uint8), o4, stream)
+        self.forward(q, k, v, np.ones(d.H, np.uint8), o16, stream)
+        sums = torch.empty(d.B * d.H * 2, dtype=torch.float64, device=self.device)
+        _check(rota_attn_head_error(d, o4, o16, sums, stream), "rota_attn_head_error")
+        _check(rota_attn_get_error(stream), "calibration")
+        st, flags, rel = rota_attn_select_fp16_heads(sums.cpu().numpy(), d.B, d.H, max_rel_err, max_fp16_heads)
+        _check(st, "rota_attn_select_fp16_heads")
+        return flags, rel
 
     def close(self):
         """Releases the copy pipeline of forward_host (if one was made)."""
