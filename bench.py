@@ -152,7 +152,7 @@ def oracle_sample(w, q, k, v, rows: int = 128):
     h = 0
     qs, ks, vs = (np.ascontiguousarray(x[:1, h:h + 1]) for x in (q, k, v))
     t0 = time.perf_counter()
-    prep = oracle.prepare(qs, ks, vs, w.grid, w.rope_dim, w.had_block, w.theta, flags)
+    prep = oracle.prepare(qs, ks, vs, w.grid, w.rope_dim, w.had_block, w.theta, flags, phase=w.rope_phase)
     t1 = time.perf_counter()
     r0 = max(0, w.N // 2 - rows // 2)
     oracle.attn_int4(prep, w.N, float(np.float32(1 / np.sqrt(w.d))), 0, 0, r0, rows)
@@ -235,7 +235,7 @@ def main():
     flags = w.flags()
     qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
     qd, kd, vd = (x.to(dev) for x in (qh, kh, vh))
-    desc = ra.make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta)
+    desc = ra.make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta, rope_phase=w.rope_phase)
     att = ra.RotaAttention(desc, device=dev, need_fp16=bool(flags.any()))
     out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device=dev)
     out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()

@@ -57,6 +57,11 @@ typedef enum {
  *   partition: a power of two (1 = no rotation) dividing rope_dim[a], <= 64.
  * rope_theta: RoPE base (10000).
  * sm_scale: softmax scale; 0 selects 1/sqrt(head_dim) (rounded to fp32).
+ * rope_phase: per partition, an angle (radians, finite) added to every pair's
+ *   RoPE angle: the "mergeable rotation fused into RoPE" of the abstract (a
+ *   fixed 2-D rotation of each pair, the rotations that commute with RoPE),
+ *   applied to Q and K alike and free at run time (it lives in the tables).
+ *   0 = plain RoPE.  It composes with had_block (rotation after RoPE).
  * head_dim: 64 or 128.
  */
 typedef struct {
@@ -66,6 +71,7 @@ typedef struct {
   int32_t had_block[3];
   float rope_theta;
   float sm_scale;
+  float rope_phase[3];
 } rota_attn_desc;
 
 /*

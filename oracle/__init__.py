@@ -51,7 +51,7 @@ def lib():
         L.oracle_float_to_half.restype = ctypes.c_uint16
         L.oracle_rope_table_len.argtypes = [P, P]
         L.oracle_rope_table_len.restype = i64
-        L.oracle_rope_tables.argtypes = [P, P, f64, P, P]
+        L.oracle_rope_tables.argtypes = [P, P, f64, P, P, P]
         L.oracle_rope_tables.restype = None
         L.oracle_rope_rotate_row.argtypes = [P, P, i64, P, P, P, P, P, i32, i32]
         L.oracle_rope_rotate_row.restype = None
@@ -65,7 +65,7 @@ def lib():
         L.oracle_code_at.restype = i32
         L.oracle_quant_codes.argtypes = [P, i64, f32, P]
         L.oracle_quant_codes.restype = None
-        L.oracle_prepare.argtypes = [i32, i32, i32, i32, P, P, P, f64] + [P] * 12
+        L.oracle_prepare.argtypes = [i32, i32, i32, i32, P, P, P, f64, P] + [P] * 12
         L.oracle_prepare.restype = i32
         L.oracle_pcode.argtypes = [f32, P]
         L.oracle_pcode.restype = i32
@@ -76,7 +76,7 @@ def lib():
         L.oracle_attn_int4.restype = i32
         L.oracle_attn_fp16.argtypes = [i32, i32, i32, i32, f32, P, P, P, i32, i32, i32, i32, P]
         L.oracle_attn_fp16.restype = i32
-        L.oracle_attn_ref.argtypes = [i32, i32, i32, i32, P, P, f64, f32, P, P, P,
+        L.oracle_attn_ref.argtypes = [i32, i32, i32, i32, P, P, f64, P, f32, P, P, P,
                                       i32, i32, i32, i32, P]
         L.oracle_attn_ref.restype = i32
         _lib = L
@@ -148,21 +148,27 @@ def quant_codes(y: np.ndarray, inv: float) -> np.ndarray:
 
 # ------------------------------------------------------------------- RoPE ---
 
-def rope_tables(grid, rope_dim, theta: float = 10000.0):
+def _phase(phase) -> np.ndarray:
+    """Per-partition RoPE phase as the library stores it (fp32), widened to double."""
+    return np.ascontiguousarray(np.asarray(phase, np.float32).astype(np.float64).reshape(3))
+
+
+def rope_tables(grid, rope_dim, theta: float = 10000.0, phase=(0.0, 0.0, 0.0)):
     g, r = _i3(grid), _i3(rope_dim)
     n = lib().oracle_rope_table_len(_p(g), _p(r))
     c = np.empty(n, np.float32)
     s = np.empty(n, np.float32)
-    lib().oracle_rope_tables(_p(g), _p(r), float(theta), _p(c), _p(s))
+    ph = _phase(phase)
+    lib().oracle_rope_tables(_p(g), _p(r), float(theta), _p(ph), _p(c), _p(s))
     return c, s
 
 
 def rope_rotate_row(x: np.ndarray, n: int, grid, rope_dim, had_block, theta: float = 10000.0,
-                    rope: bool = True, rotate: bool = True) -> np.ndarray:
+                    rope: bool = True, rotate: bool = True, phase=(0.0, 0.0, 0.0)) -> np.ndarray:
     """RoPE (token index n) then the block Hadamard rotation on one fp32 row."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     y = np.empty_like(x)
-    c, s = rope_tables(grid, rope_dim, theta)
+    c, s = rope_tables(grid, rope_dim, theta, phase)
     g, r, hb = _i3(grid), _i3(rope_dim), _i3(had_block)
     lib().oracle_rope_rotate_row(_p(x), _p(y), int(n), _p(g), _p(r), _p(hb), _p(c), _p(s),
                                  int(rope), int(rotate))
@@ -171,10 +177,11 @@ def rope_rotate_row(x: np.ndarray, n: int, grid, rope_dim, had_block, theta: flo
 
 # --------------------------------------------------------------- pipeline ---
 
-def prepare(q, k, v, grid, rope_dim, had_block, theta=10000.0, flags=None):
+def prepare(q, k, v, grid, rope_dim, had_block, theta=10000.0, flags=None, phase=(0.0, 0.0, 0.0)):
     """The prologue: returns a dict of the library-layout buffers.
 
     q, k, v: fp16 [B,H,N,d].  flags: uint8 [H] (1 = FP16 fallback head).
+    phase: per-partition RoPE phase (the merged rotation; 0 = plain RoPE).
     """
     q, k, v = _h(q), _h(k), _h(v)
     B, H, N, d = q.shape
@@ -192,7 +199,8 @@ def prepare(q, k, v, grid, rope_dim, had_block, theta=10000.0, flags=None):
         k_rope=np.zeros((B, H, N, d), np.uint16),
     )
     g, r, hb = _i3(grid), _i3(rope_dim), _i3(had_block)
-    rc = lib().oracle_prepare(B, H, N, d, _p(g), _p(r), _p(hb), float(theta),
+    ph = _phase(phase)
+    rc = lib().oracle_prepare(B, H, N, d, _p(g), _p(r), _p(hb), float(theta), _p(ph),
                               _p(q), _p(k), _p(v), _p(flags),
                               _p(out["q_codes"]), _p(out["k_codes"]), _p(out["q_scale"]),
                               _p(out["k_scale"]), _p(out["v_codes"]), _p(out["v_scale"]),
@@ -232,13 +240,14 @@ def attn_fp16(q_rope, k_rope, v, sm_scale: float, b: int, h: int, r0: int, nr: i
 
 
 def attn_ref(q, k, v, grid, rope_dim, sm_scale: float, b: int, h: int, r0: int, nr: int,
-             theta: float = 10000.0):
+             theta: float = 10000.0, phase=(0.0, 0.0, 0.0)):
     """Unquantised attention (RoPE, no rotation, double softmax) for the report."""
     q, k, v = _h(q), _h(k), _h(v)
     B, H, N, d = q.shape
     out = np.zeros((nr, d), np.float64)
     g, r = _i3(grid), _i3(rope_dim)
-    lib().oracle_attn_ref(B, H, N, d, _p(g), _p(r), float(theta), float(sm_scale),
+    ph = _phase(phase)
+    lib().oracle_attn_ref(B, H, N, d, _p(g), _p(r), float(theta), _p(ph), float(sm_scale),
                           _p(q), _p(k), _p(v), b, h, r0, nr, _p(out))
     return out
 

@@ -80,6 +80,12 @@ uint16_t oracle_float_to_half(float f)
 /* angle are evaluated in double, cos/sin in double (libm), then rounded    */
 /* to fp32.  Table layout: axis t, then h, then w; inside an axis          */
 /* [pos][pair].                                                            */
+/* The "mergeable rotation matrices that can be fused into RoPE" of the     */
+/* abstract: within a partition (distinct frequencies) the rotations that   */
+/* commute with RoPE at every position are the fixed 2-D rotations of each  */
+/* pair, so the plainest reading is one angle phase[a] per partition added  */
+/* to every pair's angle, pos * omega + phase[a] (0 = plain RoPE).  Applied */
+/* to Q and K alike it cancels in every q.k.                                */
 /* ----------------------------------------------------------------------- */
 
 static long rope_table_len(const int grid[3], const int rope_dim[3])
@@ -93,7 +99,7 @@ long oracle_rope_table_len(const int grid[3], const int rope_dim[3])
     return rope_table_len(grid, rope_dim);
 }
 
-void oracle_rope_tables(const int grid[3], const int rope_dim[3], double theta,
+void oracle_rope_tables(const int grid[3], const int rope_dim[3], double theta, const double phase[3],
                         float *cos_tab, float *sin_tab)
 {
     long off = 0;
@@ -103,7 +109,7 @@ void oracle_rope_tables(const int grid[3], const int rope_dim[3], double theta,
             for (int i = 0; i < half; ++i) {
                 double expo = -(double)(2 * i) / (double)rope_dim[a];
                 double omega = pow(theta, expo);
-                double ang = (double)pos * omega;
+                double ang = (double)pos * omega + phase[a];
                 cos_tab[off + (long)pos * half + i] = (float)cos(ang);
                 sin_tab[off + (long)pos * half + i] = (float)sin(ang);
             }
@@ -259,7 +265,7 @@ void oracle_quant_codes(const float *y, long n, float inv, int8_t *codes)
 /* ----------------------------------------------------------------------- */
 
 int oracle_prepare(int B, int H, int N, int d, const int grid[3], const int rope_dim[3],
-                   const int had_block[3], double theta,
+                   const int had_block[3], double theta, const double phase[3],
                    const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint8_t *flags,
                    uint8_t *q_codes, uint8_t *k_codes, float *q_scale, float *k_scale,
                    uint8_t *v_codes, float *v_scale, uint16_t *q_rope, uint16_t *k_rope)
@@ -274,7 +280,7 @@ int oracle_prepare(int B, int H, int N, int d, const int grid[3], const int rope
     float *blk = (float *)malloc(sizeof(float) * (size_t)QB * d);
     int *codes = (int *)malloc(sizeof(int) * (size_t)(d > QB ? d : QB));
     if (!cos_tab || !sin_tab || !x || !blk || !codes) return -1;
-    oracle_rope_tables(grid, rope_dim, theta, cos_tab, sin_tab);
+    oracle_rope_tables(grid, rope_dim, theta, phase, cos_tab, sin_tab);
 
     for (int b = 0; b < B; ++b) {
         for (int h = 0; h < H; ++h) {
@@ -528,7 +534,7 @@ int oracle_attn_fp16(int B, int H, int N, int d, float sm_scale,
 /* ----------------------------------------------------------------------- */
 
 int oracle_attn_ref(int B, int H, int N, int d, const int grid[3], const int rope_dim[3],
-                    double theta, float sm_scale, const uint16_t *q, const uint16_t *k,
+                    double theta, const double phase[3], float sm_scale, const uint16_t *q, const uint16_t *k,
                     const uint16_t *v, int b, int h, int r0, int nr, double *out)
 {
     (void)B;
@@ -540,7 +546,7 @@ int oracle_attn_ref(int B, int H, int N, int d, const int grid[3], const int rop
     double *s = (double *)malloc(sizeof(double) * (size_t)N);
     float x[1024], qr[1024];
     if (!cos_tab || !sin_tab || !kr || !s) return -1;
-    oracle_rope_tables(grid, rope_dim, theta, cos_tab, sin_tab);
+    oracle_rope_tables(grid, rope_dim, theta, phase, cos_tab, sin_tab);
     const uint16_t *qh = q + head * N * d, *kh = k + head * N * d, *vh = v + head * N * d;
     for (long kk = 0; kk < N; ++kk) {
         for (int c = 0; c < d; ++c) x[c] = oracle_half_to_float(kh[kk * d + c]);

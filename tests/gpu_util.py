@@ -16,7 +16,7 @@ def lib():
 
 
 def desc_of(w: synth.Workload):
-    return lib().make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta)
+    return lib().make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta, rope_phase=w.rope_phase)
 
 
 def to_dev(a: np.ndarray):

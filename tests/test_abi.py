@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(ra):
 
 
 def _desc(ra, w):
-    return ra.make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta)
+    return ra.make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta, rope_phase=w.rope_phase)
 
 
 def test_validate_accepts_workloads(ra):
@@ -92,11 +92,14 @@ def test_buffer_sizes(ra):
     assert sz[ra.ROTA_BUF_ROPE_TABLE] == 4 * (21 * 22 + 30 * 21 + 52 * 21)
 
 
-@pytest.mark.parametrize("name", ["tiny", "wan480", "wan720", "hunyuan"])
+@pytest.mark.parametrize("name", ["tiny", "wan480", "wan720", "hunyuan", "wan480_phase"])
 def test_rope_tables_identical_to_oracle(ra, name):
-    w = synth.WORKLOADS[name]
+    if name == "wan480_phase":   # the merged per-pair rotation: a phase per partition
+        w = synth.scaled(synth.WORKLOADS["wan480"], name, rope_phase=(0.3, 0.7853982, -2.5))
+    else:
+        w = synth.WORKLOADS[name]
     c, s = ra.rota_attn_build_rope_tables(_desc(ra, w))
-    oc, os_ = oracle.rope_tables(w.grid, w.rope_dim, w.theta)
+    oc, os_ = oracle.rope_tables(w.grid, w.rope_dim, w.theta, w.rope_phase)
     assert np.array_equal(c.view(np.uint32), oc.view(np.uint32))
     assert np.array_equal(s.view(np.uint32), os_.view(np.uint32))
 

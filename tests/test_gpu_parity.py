@@ -4,6 +4,8 @@ Bars: integer codes, scales, RoPE'd fp16 rows, s32 scores and P codes
 bit-exact; attention outputs within max-abs 2e-3 of the oracle's double
 result.  Sizes span several 128-row tiles and 64-key blocks with a ragged
 tail (N mod 64 != 0), both head dims (64, 128) and all three RoPE splits."""
+import math
+
 import numpy as np
 import pytest
 
@@ -25,6 +27,10 @@ CASES = {
     "offgrid": synth.scaled(synth.WORKLOADS["wan480"], "offgrid", H=2, grid=(2, 7, 11), rope_dim=(42, 44, 42)),
     # rotation blocks of 32 and 64 channels (the largest Hadamard orders)
     "wide_blocks": synth.scaled(synth.WORKLOADS["wan480"], "wide", H=1, grid=(2, 5, 7), rope_dim=(32, 32, 64)),
+    # the merged per-pair rotation (a phase in the RoPE tables) in place of the 2-channel
+    # Hadamard blocks of the h and w partitions, and on top of the 4-channel ones of t
+    "merged_phase": synth.scaled(synth.WORKLOADS["wan480"], "merged", H=2, grid=(3, 10, 13), had=(4, 1, 1),
+                                 rope_phase=(0.3, math.pi / 4, -math.pi / 4)),
 }
 
 # Many key blocks per CTA (74), so every pipeline stage and barrier phase wraps many times.
@@ -32,7 +38,7 @@ LONG = synth.scaled(synth.WORKLOADS["wan480"], "wan_long", H=2, grid=(3, 30, 52)
 
 
 def _oracle(w, q, k, v, flags=None):
-    return oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block, w.theta, flags)
+    return oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block, w.theta, flags, phase=w.rope_phase)
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -74,7 +80,7 @@ def test_int4_output_all_heads(name):
         assert e <= TOL, (h, e, rel, cos)
 
 
-@pytest.mark.parametrize("name", ["tiny", "wan_mini", "ragged_small"])
+@pytest.mark.parametrize("name", ["tiny", "wan_mini", "ragged_small", "merged_phase"])
 def test_fp16_fallback_heads(name):
     w = CASES[name]
     q, k, v = synth.make_inputs(w)

@@ -126,6 +126,44 @@ def test_rope_identity_at_origin_and_relative_position():
         assert abs(a - b) < 1e-4 * (1 + abs(a))
 
 
+def _pair_rotate(y: np.ndarray, rope_dim, phase) -> np.ndarray:
+    """Rotate every RoPE pair (2i, 2i+1) of partition a by phase[a], in double."""
+    out = y.astype(np.float64).copy()
+    c0 = 0
+    for a, da in enumerate(rope_dim):
+        ph = float(np.float32(phase[a]))
+        c, s = math.cos(ph), math.sin(ph)
+        for i in range(c0, c0 + da, 2):
+            x0, x1 = out[i], out[i + 1]
+            out[i], out[i + 1] = c * x0 - s * x1, s * x0 + c * x1
+        c0 += da
+    return out
+
+
+@pytest.mark.parametrize("phase", [(0.3, math.pi / 4, -math.pi / 4), (-2.5, 1.0, 3.0)])
+def test_merged_rotation_is_rope_then_pair_rotation(phase):
+    """The phase in the tables equals RoPE followed by a fixed rotation of each
+    pair (closed form in double; the tables' fp32 rounding is the only gap), is
+    the pure pair rotation at position 0, and cancels in q.k (same phase on Q
+    and K) up to that rounding."""
+    rope_dim, grid = (44, 42, 42), (3, 5, 7)
+    rng = np.random.default_rng(13)
+    q = rng.standard_normal(128).astype(np.float32)
+    k = rng.standard_normal(128).astype(np.float32)
+    for n in (0, 17, 104):
+        yp = oracle.rope_rotate_row(q, n, grid, rope_dim, (1, 1, 1), rotate=False, phase=phase)
+        y0 = oracle.rope_rotate_row(q, n, grid, rope_dim, (1, 1, 1), rotate=False)
+        assert np.abs(yp - _pair_rotate(y0, rope_dim, phase)).max() < 1e-5 * np.abs(q).max()
+    y = oracle.rope_rotate_row(q, 0, grid, rope_dim, (1, 1, 1), rotate=False, phase=phase)
+    assert np.abs(y - _pair_rotate(q, rope_dim, phase)).max() < 1e-6 * np.abs(q).max()
+    for n1, n2 in ((0, 0), (5, 77), (104, 3)):
+        a = np.dot(oracle.rope_rotate_row(q, n1, grid, rope_dim, (1, 1, 1), rotate=False, phase=phase).astype(np.float64),
+                   oracle.rope_rotate_row(k, n2, grid, rope_dim, (1, 1, 1), rotate=False, phase=phase))
+        b = np.dot(oracle.rope_rotate_row(q, n1, grid, rope_dim, (1, 1, 1), rotate=False).astype(np.float64),
+                   oracle.rope_rotate_row(k, n2, grid, rope_dim, (1, 1, 1), rotate=False))
+        assert abs(a - b) < 1e-4 * (1 + abs(b))
+
+
 # -------------------------------------------------------------- rotation ---
 
 @pytest.mark.parametrize("rope_dim,had", [((16, 24, 24), (16, 8, 8)), ((44, 42, 42), (4, 2, 2)),

@@ -197,6 +197,8 @@ rota_status rota_attn_validate(const rota_attn_desc* d) {
   if (sum != d->head_dim) return ROTA_ERR_INVALID_ARG;
   if (!(d->rope_theta > 0.f) || !std::isfinite(d->rope_theta)) return ROTA_ERR_INVALID_ARG;
   if (!(d->sm_scale >= 0.f) || !std::isfinite(d->sm_scale)) return ROTA_ERR_INVALID_ARG;
+  for (int a = 0; a < 3; ++a)
+    if (!std::isfinite(d->rope_phase[a])) return ROTA_ERR_INVALID_ARG;
   if (d->head_dim != 64 && d->head_dim != 128) return ROTA_ERR_UNSUPPORTED;
   if (d->H > 256) return ROTA_ERR_UNSUPPORTED;
   if (static_cast<long long>(d->B) * d->H * npad_of(d->N) * d->head_dim > (1ll << 40)) return ROTA_ERR_UNSUPPORTED;
@@ -234,11 +236,12 @@ rota_status rota_attn_build_rope_tables(const rota_attn_desc* d, float* host_cos
   size_t base = 0;
   for (int a = 0; a < 3; ++a) {
     const int half = d->rope_dim[a] / 2;
+    const double phase = static_cast<double>(d->rope_phase[a]);   // the merged per-pair rotation
     for (int i = 0; i < half; ++i) {
       // omega_i = theta^(-2i / d_a), evaluated in double
       const double omega = std::pow(theta, -static_cast<double>(2 * i) / static_cast<double>(d->rope_dim[a]));
       for (int pos = 0; pos < extent[a]; ++pos) {
-        const double angle = static_cast<double>(pos) * omega;
+        const double angle = static_cast<double>(pos) * omega + phase;
         host_cos[base + static_cast<size_t>(pos) * half + i] = static_cast<float>(std::cos(angle));
         host_sin[base + static_cast<size_t>(pos) * half + i] = static_cast<float>(std::sin(angle));
       }

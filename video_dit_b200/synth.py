@@ -46,6 +46,10 @@ class Workload:
     v_token_scale: float = 1.0
     fp16_every: int = 0          # heads h with h % fp16_every == 0 take the FP16 fallback
     all_fp16: bool = False
+    # rotation: Hadamard block per partition (None = the default block) and the
+    # merged per-pair rotation angle added to every RoPE angle (0 = plain RoPE)
+    had: Optional[Tuple[int, int, int]] = None
+    rope_phase: Tuple[float, float, float] = (0.0, 0.0, 0.0)
 
     @property
     def N(self) -> int:
@@ -53,6 +57,8 @@ class Workload:
 
     @property
     def had_block(self) -> Tuple[int, int, int]:
+        if self.had is not None:
+            return tuple(self.had)
         return tuple(default_had_block(r) for r in self.rope_dim)
 
     def flags(self) -> np.ndarray:
