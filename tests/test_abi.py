@@ -215,3 +215,13 @@ def test_select_rejects_null_pointers(ra):
     flags = np.zeros(4, np.uint8)
     assert ra._lib.rota_attn_select_fp16_heads(None, 1, 4, 0.1, -1, None, flags.ctypes.data) == ra.ROTA_ERR_INVALID_ARG
     assert ra._lib.rota_attn_select_fp16_heads(s.ctypes.data, 1, 4, 0.1, -1, None, None) == ra.ROTA_ERR_INVALID_ARG
+
+
+def test_validate_rejects_non_finite_phase(ra):
+    d = _desc(ra, synth.WORKLOADS["wan480"])
+    d.rope_phase[1] = float("inf")
+    assert ra.rota_attn_validate(d) == ra.ROTA_ERR_INVALID_ARG
+    d.rope_phase[1] = float("nan")
+    assert ra.rota_attn_validate(d) == ra.ROTA_ERR_INVALID_ARG
+    d.rope_phase[1] = -3.0
+    assert ra.rota_attn_validate(d) == ra.ROTA_OK
