@@ -79,6 +79,8 @@ def lib():
         L.oracle_attn_ref.argtypes = [i32, i32, i32, i32, P, P, f64, P, f32, P, P, P,
                                       i32, i32, i32, i32, P]
         L.oracle_attn_ref.restype = i32
+        L.oracle_hadamard.argtypes = [i32, P]
+        L.oracle_hadamard.restype = i32
         _lib = L
     return _lib
 
@@ -161,6 +163,14 @@ def rope_tables(grid, rope_dim, theta: float = 10000.0, phase=(0.0, 0.0, 0.0)):
     ph = _phase(phase)
     lib().oracle_rope_tables(_p(g), _p(r), float(theta), _p(ph), _p(c), _p(s))
     return c, s
+
+
+def hadamard(n: int):
+    """The oracle's Hadamard matrix of a non-power-of-two order n (int8 +1/-1,
+    n x n), or None if it builds none of that order."""
+    h = np.zeros((n, n), np.int8) if n > 0 else np.zeros((1, 1), np.int8)
+    ok = lib().oracle_hadamard(int(n), _p(h))
+    return h if ok else None
 
 
 def rope_rotate_row(x: np.ndarray, n: int, grid, rope_dim, had_block, theta: float = 10000.0,

@@ -163,12 +163,127 @@ static void rope_row(const float *x, float *y, long n, const int grid[3], const 
 /* Q K^T is unchanged in exact arithmetic; V is not rotated.               */
 /* ----------------------------------------------------------------------- */
 
+/* Blocks whose size is not a power of two (the survey's numerics variant:  */
+/* the partition's own size, e.g. 44 for a 44-channel partition) take a     */
+/* Hadamard matrix of that order from the classical constructions:          */
+/*   Paley I  (q prime, q = 3 mod 4), order q + 1:  H = I + S,             */
+/*            S = [[0, 1^T], [-1, Q]],  Q_ij = chi(j - i);                  */
+/*   Paley II (q prime, q = 1 mod 4), order 2(q + 1):  from the conference */
+/*            matrix C = [[0, 1^T], [1, Q]], every off-diagonal entry c ->  */
+/*            c [[1, 1], [1, -1]], every diagonal entry -> [[1, -1], [-1, -1]];*/
+/*   doubling: H_2n = [[H, H], [H, -H]].                                   */
+/* chi is the quadratic character mod q (chi(0) = 0).  For an order n <= 64 */
+/* that is not a power of two the first rule that applies is used:          */
+/* doubling (n / 2 >= 12 and supported), Paley I (q = n - 1), Paley II      */
+/* (q = n / 2 - 1); e.g. 12, 20, 44, 60 by Paley I (q = 11, 19, 43, 59),    */
+/* 28, 36 by Paley II (q = 13, 17), 24, 40, 48, 56 by doubling.  Other     */
+/* orders (6, 10, 14, ...) are unsupported.  Such a block is applied as a dense */
+/* product, y_i = sum_j H_ij x_j accumulated in fp32 in the order          */
+/* j = 0, 1, ..., b-1 (the first term exact, then one add or subtract per  */
+/* term), then y_i * r_b.                                                  */
+static int chi(long a, int q)
+{
+    a %= q;
+    if (a < 0) a += q;
+    if (a == 0) return 0;
+    long r = 1, base = a, e = (q - 1) / 2;
+    while (e > 0) {
+        if (e & 1) r = r * base % q;
+        base = base * base % q;
+        e >>= 1;
+    }
+    return r == 1 ? 1 : -1;
+}
+
+static int is_prime(int q)
+{
+    if (q < 2) return 0;
+    for (int f = 2; f * f <= q; ++f)
+        if (q % f == 0) return 0;
+    return 1;
+}
+
+/* H (n x n, row-major, entries +1 / -1) for a supported non-power-of-two    */
+/* order n <= 64; returns 0 for any other n.                                */
+int oracle_hadamard(int n, signed char *H)
+{
+    if (n <= 1 || n > 64 || (n & (n - 1)) == 0) return 0;
+    if (n % 2 == 0 && n / 2 >= 12 && oracle_hadamard(n / 2, NULL)) {
+        if (H) {
+            int m = n / 2;
+            signed char *h = (signed char *)malloc((size_t)m * m);
+            if (!h) return 0;
+            oracle_hadamard(m, h);
+            for (int i = 0; i < m; ++i)
+                for (int j = 0; j < m; ++j) {
+                    H[i * n + j] = h[i * m + j];
+                    H[i * n + j + m] = h[i * m + j];
+                    H[(i + m) * n + j] = h[i * m + j];
+                    H[(i + m) * n + j + m] = (signed char)-h[i * m + j];
+                }
+            free(h);
+        }
+        return 1;
+    }
+    int q = n - 1;
+    if (q % 4 == 3 && is_prime(q)) {           /* Paley I */
+        if (H)
+            for (int i = 0; i < n; ++i)
+                for (int j = 0; j < n; ++j) {
+                    int sv;
+                    if (i == j) sv = 1;                      /* I + S, S_ii = 0 */
+                    else if (i == 0) sv = 1;                 /* first row of S: 1 */
+                    else if (j == 0) sv = -1;                /* first column of S: -1 */
+                    else sv = chi((long)(j - 1) - (i - 1), q);
+                    H[i * n + j] = (signed char)sv;
+                }
+        return 1;
+    }
+    if (n % 2 == 0) {
+        q = n / 2 - 1;
+        if (q % 4 == 1 && is_prime(q)) {       /* Paley II */
+            if (H) {
+                int m = q + 1;
+                for (int i = 0; i < m; ++i)
+                    for (int j = 0; j < m; ++j) {
+                        int c;
+                        if (i == j) c = 0;
+                        else if (i == 0 || j == 0) c = 1;
+                        else c = chi((long)(j - 1) - (i - 1), q);
+                        int e00, e01, e10, e11;
+                        if (c == 0) { e00 = 1; e01 = -1; e10 = -1; e11 = -1; }
+                        else { e00 = c; e01 = c; e10 = c; e11 = -c; }
+                        H[(2 * i) * n + 2 * j] = (signed char)e00;
+                        H[(2 * i) * n + 2 * j + 1] = (signed char)e01;
+                        H[(2 * i + 1) * n + 2 * j] = (signed char)e10;
+                        H[(2 * i + 1) * n + 2 * j + 1] = (signed char)e11;
+                    }
+            }
+            return 1;
+        }
+    }
+    return 0;
+}
+
 static void rotate_row(float *y, const int rope_dim[3], const int had_block[3])
 {
     int coff = 0;
     for (int a = 0; a < 3; ++a) {
         int b = had_block[a];
-        if (b > 1) {
+        if (b > 1 && (b & (b - 1)) != 0) {       /* dense block of a non-power-of-two order */
+            float r = (float)(1.0 / sqrt((double)b));
+            signed char H[64 * 64];
+            float t[64];
+            if (!oracle_hadamard(b, H)) { coff += rope_dim[a]; continue; }
+            for (int blk = coff; blk < coff + rope_dim[a]; blk += b) {
+                for (int i = 0; i < b; ++i) {
+                    float acc = H[i * b] > 0 ? y[blk] : -y[blk];
+                    for (int j = 1; j < b; ++j) acc = H[i * b + j] > 0 ? acc + y[blk + j] : acc - y[blk + j];
+                    t[i] = acc;
+                }
+                for (int i = 0; i < b; ++i) y[blk + i] = t[i] * r;
+            }
+        } else if (b > 1) {
             float r = (float)(1.0 / sqrt((double)b));
             for (int blk = coff; blk < coff + rope_dim[a]; blk += b) {
                 for (int h = 1; h < b; h <<= 1) {

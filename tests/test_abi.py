@@ -225,3 +225,18 @@ def test_validate_rejects_non_finite_phase(ra):
     assert ra.rota_attn_validate(d) == ra.ROTA_ERR_INVALID_ARG
     d.rope_phase[1] = -3.0
     assert ra.rota_attn_validate(d) == ra.ROTA_OK
+
+
+@pytest.mark.parametrize("had,ok", [((44, 2, 2), True), ((4, 42, 42), False), ((12, 2, 2), False),
+                                    ((44, 6, 2), False), ((4, 14, 14), False)])
+def test_validate_hadamard_orders(ra, had, ok):
+    # 44 = Paley I (q = 43); 42 and 14 (which divide 42) and 6 are orders with no
+    # Hadamard matrix; 12 is one but does not divide 44
+    d = _desc(ra, synth.scaled(synth.WORKLOADS["wan480"], "v", had=had))
+    assert ra.rota_attn_validate(d) == (ra.ROTA_OK if ok else ra.ROTA_ERR_INVALID_ARG)
+
+
+@pytest.mark.parametrize("had", [(16, 56, 56), (16, 28, 28), (16, 8, 8)])
+def test_validate_hunyuan_orders(ra, had):
+    d = _desc(ra, synth.scaled(synth.WORKLOADS["hunyuan"], "v", had=had))
+    assert ra.rota_attn_validate(d) == ra.ROTA_OK

@@ -31,6 +31,10 @@ CASES = {
     # Hadamard blocks of the h and w partitions, and on top of the 4-channel ones of t
     "merged_phase": synth.scaled(synth.WORKLOADS["wan480"], "merged", H=2, grid=(3, 10, 13), had=(4, 1, 1),
                                  rope_phase=(0.3, math.pi / 4, -math.pi / 4)),
+    # Hadamard blocks of non-power-of-two orders: the whole 44-channel partition (Paley I,
+    # q = 43) and the 56-channel ones (Paley II, q = 13, doubled)
+    "hadamard_44": synth.scaled(synth.WORKLOADS["wan480"], "h44", H=2, grid=(3, 10, 13), had=(44, 2, 2)),
+    "hadamard_56": synth.scaled(synth.WORKLOADS["hunyuan"], "h56", H=2, grid=(3, 9, 20), had=(16, 56, 56)),
 }
 
 # Many key blocks per CTA (74), so every pipeline stage and barrier phase wraps many times.

@@ -182,6 +182,53 @@ def test_rotation_is_blockdiag_sylvester_hadamard(rope_dim, had):
     assert np.abs(M @ M.T - np.eye(d)).max() < 1e-6
 
 
+@pytest.mark.parametrize("n", [12, 20, 24, 28, 36, 40, 44, 48, 56, 60])
+def test_nonpow2_hadamard_is_hadamard(n):
+    """H H^T = n I exactly, entries +-1 (the definition of a Hadamard matrix)."""
+    h = oracle.hadamard(n)
+    assert h is not None
+    assert set(np.unique(h).tolist()) == {-1, 1}
+    assert np.array_equal(h.astype(np.int64) @ h.T.astype(np.int64), n * np.eye(n, dtype=np.int64))
+
+
+@pytest.mark.parametrize("n", [6, 10, 14, 18, 22, 52])
+def test_nonpow2_hadamard_unsupported_orders(n):
+    # 2 mod 4 orders > 2 admit no Hadamard matrix; 52 is none of the three constructions
+    assert oracle.hadamard(n) is None
+
+
+@pytest.mark.parametrize("rope_dim,had", [((44, 42, 42), (44, 2, 2)), ((16, 56, 56), (16, 56, 56)),
+                                          ((24, 20, 20), (12, 20, 20))])
+def test_dense_rotation_is_normalised_hadamard_and_keeps_qk(rope_dim, had):
+    """A non-power-of-two block is the dense product (H / sqrt(b)) x (checked in
+    double against the matrix), and q.k is unchanged by it."""
+    grid = (2, 3, 5)
+    d = sum(rope_dim)
+    rng = np.random.default_rng(17)
+    q = rng.standard_normal(d).astype(np.float32)
+    k = rng.standard_normal(d).astype(np.float32)
+    yq = oracle.rope_rotate_row(q, 7, grid, rope_dim, had)
+    y0 = oracle.rope_rotate_row(q, 7, grid, rope_dim, (1, 1, 1), rotate=True)
+    # the expected rotation, block by block, in double
+    want = y0.astype(np.float64).copy()
+    c0 = 0
+    for a, (da, b) in enumerate(zip(rope_dim, had)):
+        if b > 1:
+            m = oracle.hadamard(b) if b & (b - 1) else None
+            if m is None:
+                from scipy.linalg import hadamard as sylvester
+                m = sylvester(b)
+            for blk in range(c0, c0 + da, b):
+                want[blk:blk + b] = (m.astype(np.float64) @ want[blk:blk + b]) / math.sqrt(b)
+        c0 += da
+    assert np.abs(yq - want).max() < 1e-5 * np.abs(want).max()
+    yk = oracle.rope_rotate_row(k, 11, grid, rope_dim, had)
+    zk = oracle.rope_rotate_row(k, 11, grid, rope_dim, (1, 1, 1), rotate=True)
+    a = float(np.dot(yq.astype(np.float64), yk))
+    b = float(np.dot(y0.astype(np.float64), zk))
+    assert abs(a - b) < 1e-4 * (1 + abs(b))
+
+
 def test_rotation_preserves_qk():
     rope_dim, had = (44, 42, 42), (4, 2, 2)
     rng = np.random.default_rng(3)

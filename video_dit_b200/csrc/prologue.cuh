@@ -39,6 +39,8 @@ struct PrologueParams {
                      // (no rotation, or had[a] <= 8 and coff[a] % had[a] == 0: every
                      // unit then lies inside one 8-channel chunk)
   int any_unfused;   // some partition needs the shared-memory rotation pass
+  int dense[3];      // partition a's block is not a power of two: a dense Hadamard product
+  uint64_t hneg[3][64];  // its rows: bit j of row i set where H_ij = -1
   int coff[3];       // channel offset of each partition
   int toff[3];       // table offset of each axis
   float rnorm[3];    // RN(1 / sqrt(had[a]))
@@ -108,6 +110,27 @@ __device__ __noinline__ float rotate_unit_smem(float* xrow, int c0, int G, float
   for (int j = 0; j < G; ++j) {
     y[j] = __fmul_rn(y[j], rnorm);
     amax = fmaxf(amax, fabsf(y[j]));
+  }
+  return amax;
+}
+
+// A rotation unit whose order is not a power of two: y_i = sum_j H_ij x_j in
+// fp32 in the order j = 0, 1, ..., G-1 (the first term exact, then one add or
+// subtract per term), then y_i * rnorm; the rows of H as sign masks.  The
+// unit's inputs are all read before any output is stored.
+__device__ __noinline__ float rotate_unit_dense(float* xrow, int c0, int G, const uint64_t* neg, float rnorm) {
+  float* x = xrow + c0;
+  float y[64];
+  for (int i = 0; i < G; ++i) {
+    const uint64_t m = neg[i];
+    float acc = (m & 1ull) ? -x[0] : x[0];
+    for (int j = 1; j < G; ++j) acc = ((m >> j) & 1ull) ? __fsub_rn(acc, x[j]) : __fadd_rn(acc, x[j]);
+    y[i] = acc;
+  }
+  float amax = 0.f;
+  for (int i = 0; i < G; ++i) {
+    x[i] = __fmul_rn(y[i], rnorm);
+    amax = fmaxf(amax, fabsf(x[i]));
   }
   return amax;
 }
@@ -184,7 +207,7 @@ __device__ __forceinline__ void load_tile(const __half* src, int n0, int N, floa
 }
 
 template <int D>
-__global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const PrologueParams p) {
+__global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const __grid_constant__ PrologueParams p) {
   constexpr int LD = D + 4;
   __shared__ __align__(16) float X[64 * LD];
   __shared__ float red[kPrologueThreads / 32];
@@ -330,11 +353,15 @@ __global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const Pro
           float* xrow = X + r * LD;
           const int c0 = p.coff[a] + un * G;
           float m;
-          switch (G) {
-            case 2: m = rotate_unit<2>(xrow, c0, p.rnorm[a]); break;
-            case 4: m = rotate_unit<4>(xrow, c0, p.rnorm[a]); break;
-            case 8: m = rotate_unit<8>(xrow, c0, p.rnorm[a]); break;
-            default: m = rotate_unit_smem(xrow, c0, G, p.rnorm[a]); break;
+          if (p.dense[a]) {
+            m = rotate_unit_dense(xrow, c0, G, p.hneg[a], p.rnorm[a]);
+          } else {
+            switch (G) {
+              case 2: m = rotate_unit<2>(xrow, c0, p.rnorm[a]); break;
+              case 4: m = rotate_unit<4>(xrow, c0, p.rnorm[a]); break;
+              case 8: m = rotate_unit<8>(xrow, c0, p.rnorm[a]); break;
+              default: m = rotate_unit_smem(xrow, c0, G, p.rnorm[a]); break;
+            }
           }
           amax = fmaxf(amax, m);
         }

@@ -79,6 +79,72 @@ rota_status set_smem(K kernel, int bytes) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Hadamard matrices of orders that are not powers of two (rows as sign masks:
+// bit j of row i set where H_ij = -1).  The first construction that applies:
+// doubling [[H, H], [H, -H]] of a supported order >= 12; Paley I for a prime
+// q = n - 1 = 3 (mod 4): H = I + [[0, 1^T], [-1, Q]]; Paley II for a prime
+// q = n / 2 - 1 = 1 (mod 4): the conference matrix [[0, 1^T], [1, Q]] with
+// every off-diagonal entry c replaced by c [[1, 1], [1, -1]] and every
+// diagonal entry by [[1, -1], [-1, -1]].  Q_ij = chi(j - i), chi the quadratic
+// character mod q.  Returns false for an unsupported order.
+int quad_char(long a, int q) {
+  a %= q;
+  if (a < 0) a += q;
+  if (a == 0) return 0;
+  long r = 1, b = a;
+  for (long e = (q - 1) / 2; e > 0; e >>= 1) {
+    if (e & 1) r = r * b % q;
+    b = b * b % q;
+  }
+  return r == 1 ? 1 : -1;
+}
+
+bool prime(int q) {
+  if (q < 2) return false;
+  for (int f = 2; f * f <= q; ++f)
+    if (q % f == 0) return false;
+  return true;
+}
+
+bool hadamard_rows(int n, uint64_t* neg) {
+  if (n <= 1 || n > 64 || is_pow2(n)) return false;
+  uint64_t half[64];
+  if (n % 2 == 0 && n / 2 >= 12 && hadamard_rows(n / 2, half)) {
+    const int m = n / 2;
+    const uint64_t lo = (m == 64) ? ~0ull : ((1ull << m) - 1);
+    for (int i = 0; i < m; ++i) {
+      neg[i] = half[i] | (half[i] << m);                  // [H, H]
+      neg[i + m] = half[i] | ((~half[i] & lo) << m);      // [H, -H]
+    }
+    return true;
+  }
+  auto put = [&](int i, int j, int v) {
+    if (v < 0) neg[i] |= 1ull << j;
+  };
+  for (int i = 0; i < n; ++i) neg[i] = 0;
+  int q = n - 1;
+  if (q % 4 == 3 && prime(q)) {
+    for (int i = 0; i < n; ++i)
+      for (int j = 0; j < n; ++j)
+        put(i, j, i == j ? 1 : i == 0 ? 1 : j == 0 ? -1 : quad_char(static_cast<long>(j) - i, q));
+    return true;
+  }
+  q = n / 2 - 1;
+  if (n % 2 == 0 && q % 4 == 1 && prime(q)) {
+    const int m = q + 1;
+    for (int i = 0; i < m; ++i)
+      for (int j = 0; j < m; ++j) {
+        const int c = i == j ? 0 : (i == 0 || j == 0) ? 1 : quad_char(static_cast<long>(j) - i, q);
+        put(2 * i, 2 * j, c == 0 ? 1 : c);
+        put(2 * i, 2 * j + 1, c == 0 ? -1 : c);
+        put(2 * i + 1, 2 * j, c == 0 ? -1 : c);
+        put(2 * i + 1, 2 * j + 1, c == 0 ? -1 : -c);
+      }
+    return true;
+  }
+  return false;
+}
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 // The buffers the INT4 path reads or writes: q_scale and k_scale are touched
@@ -190,7 +256,9 @@ rota_status rota_attn_validate(const rota_attn_desc* d) {
   int sum = 0;
   for (int a = 0; a < 3; ++a) {
     if (d->rope_dim[a] < 2 || d->rope_dim[a] % 2) return ROTA_ERR_INVALID_ARG;
-    if (!is_pow2(d->had_block[a]) || d->had_block[a] > 64 || d->rope_dim[a] % d->had_block[a])
+    uint64_t rows[64];
+    const int hb = d->had_block[a];
+    if (hb < 1 || hb > 64 || d->rope_dim[a] % hb || !(is_pow2(hb) || hadamard_rows(hb, rows)))
       return ROTA_ERR_INVALID_ARG;
     sum += d->rope_dim[a];
   }
@@ -292,6 +360,7 @@ rota_status rota_attn_prepare_qk(const rota_attn_desc* d, const uint16_t* q, con
     p.toff[a] = toff;
     p.rnorm[a] = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d->had_block[a])));
     p.fused[a] = d->had_block[a] <= 1 || (d->had_block[a] <= 8 && coff % d->had_block[a] == 0);
+    p.dense[a] = hadamard_rows(d->had_block[a], p.hneg[a]) ? 1 : 0;
     if (!p.fused[a]) p.any_unfused = 1;
     coff += d->rope_dim[a];
     toff += extent[a] * (d->rope_dim[a] / 2);

@@ -94,6 +94,10 @@ WORKLOADS = {
     "hunyuan": Workload("hunyuan", B=1, H=24, d=128, rope_dim=(16, 56, 56), grid=(33, 34, 60),
                         qk_outliers=(4, 0, 0), qk_scale=25.0),
 }
+# the rotation variants on the full-size recipes: the whole 44-channel temporal partition
+# as one Hadamard block (Paley I, q = 43) and the 56-channel ones (Paley II, q = 13, doubled)
+WORKLOADS["wan480_h44"] = dataclasses.replace(WORKLOADS["wan480"], name="wan480_h44", had=(44, 2, 2))
+WORKLOADS["hunyuan_h56"] = dataclasses.replace(WORKLOADS["hunyuan"], name="hunyuan_h56", had=(16, 56, 56))
 for _F in (3, 6, 11, 21, 31):
     WORKLOADS[f"sweep{_F}"] = Workload(f"sweep{_F}", B=1, H=40, grid=(_F, 30, 52), **_WAN)
     WORKLOADS[f"sweep{_F}_fp16"] = Workload(f"sweep{_F}_fp16", B=1, H=40, grid=(_F, 30, 52),
