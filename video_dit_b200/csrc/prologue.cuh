@@ -114,23 +114,60 @@ __device__ __noinline__ float rotate_unit_smem(float* xrow, int c0, int G, float
   return amax;
 }
 
-// A rotation unit whose order is not a power of two: y_i = sum_j H_ij x_j in
-// fp32 in the order j = 0, 1, ..., G-1 (the first term exact, then one add or
-// subtract per term), then y_i * rnorm; the rows of H as sign masks.  The
-// unit's inputs are all read before any output is stored.
-__device__ __noinline__ float rotate_unit_dense(float* xrow, int c0, int G, const uint64_t* neg, float rnorm) {
-  float* x = xrow + c0;
-  float y[64];
-  for (int i = 0; i < G; ++i) {
-    const uint64_t m = neg[i];
-    float acc = (m & 1ull) ? -x[0] : x[0];
-    for (int j = 1; j < G; ++j) acc = ((m >> j) & 1ull) ? __fsub_rn(acc, x[j]) : __fadd_rn(acc, x[j]);
-    y[i] = acc;
-  }
+// The rotation units of one partition whose order G is not a power of two,
+// by all threads of the CTA: y_i = sum_j H_ij x_j in fp32 in the order
+// j = 0, 1, ..., G-1 (the first term exact, then one add of +-x_j per term),
+// then y_i * rnorm.  One thread takes 8 output rows of one (token, unit); a
+// round holds whole (token, unit) groups, so every input of a group is read
+// before the barrier and every output stored after it.  The rows of H come as
+// sign masks (bit j of row i set where H_ij = -1).  Returns the thread's max |y|.
+template <int LD>
+__device__ float rotate_partition_dense(float* X, int c_off, int G, int d_a, const uint64_t* neg, float rnorm,
+                                        int rows) {
+  const int nch = (G + 7) >> 3;
+  const int per_round = (kPrologueThreads / nch) * nch;
+  const int njobs = 64 * (d_a / G) * nch;          // (token, unit, 8 rows), tokens fastest within a unit
   float amax = 0.f;
-  for (int i = 0; i < G; ++i) {
-    x[i] = __fmul_rn(y[i], rnorm);
-    amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll 1
+  for (int base = 0; base < njobs; base += per_round) {
+    const int job = base + static_cast<int>(threadIdx.x);
+    const bool act = static_cast<int>(threadIdx.x) < per_round && job < njobs;
+    int r = 0, c0 = 0, ch = 0;
+    float acc[8];
+    if (act) {
+      const int g = job / nch;
+      ch = job - g * nch;
+      r = g & 63;
+      c0 = c_off + (g >> 6) * G;
+      if (r < rows) {
+        const float* x = X + r * LD + c0;
+        uint64_t m[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m[k] = 8 * ch + k < G ? neg[8 * ch + k] : 0ull;
+        const float x0 = x[0];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = (m[k] & 1ull) ? -x0 : x0;
+#pragma unroll 1
+        for (int j = 1; j < G; ++j) {
+          const uint32_t xb = __float_as_uint(x[j]);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            acc[k] = __fadd_rn(acc[k], __uint_as_float(xb ^ (static_cast<uint32_t>(m[k] >> j) << 31)));
+        }
+      }
+    }
+    __syncthreads();
+    if (act && r < rows) {
+      float* x = X + r * LD + c0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (8 * ch + k < G) {
+          const float y = __fmul_rn(acc[k], rnorm);
+          x[8 * ch + k] = y;
+          amax = fmaxf(amax, fabsf(y));
+        }
+    }
+    __syncthreads();
   }
   return amax;
 }
@@ -345,6 +382,11 @@ __global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const __g
       for (int a = 0; a < 3; ++a) {
         if (p.fused[a]) continue;
         const int G = p.had[a];
+        if (p.dense[a]) {    // uniform: every thread takes part in the rounds
+          amax = fmaxf(amax, rotate_partition_dense<LD>(X, p.coff[a], G, p.rope_dim[a], p.hneg[a], p.rnorm[a],
+                                                        p.N - n0));
+          continue;
+        }
         const int njobs = 64 * (p.rope_dim[a] / G);
 #pragma unroll 1
         for (int j = threadIdx.x; j < njobs; j += kPrologueThreads) {
@@ -353,15 +395,11 @@ __global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const __g
           float* xrow = X + r * LD;
           const int c0 = p.coff[a] + un * G;
           float m;
-          if (p.dense[a]) {
-            m = rotate_unit_dense(xrow, c0, G, p.hneg[a], p.rnorm[a]);
-          } else {
-            switch (G) {
-              case 2: m = rotate_unit<2>(xrow, c0, p.rnorm[a]); break;
-              case 4: m = rotate_unit<4>(xrow, c0, p.rnorm[a]); break;
-              case 8: m = rotate_unit<8>(xrow, c0, p.rnorm[a]); break;
-              default: m = rotate_unit_smem(xrow, c0, G, p.rnorm[a]); break;
-            }
+          switch (G) {
+            case 2: m = rotate_unit<2>(xrow, c0, p.rnorm[a]); break;
+            case 4: m = rotate_unit<4>(xrow, c0, p.rnorm[a]); break;
+            case 8: m = rotate_unit<8>(xrow, c0, p.rnorm[a]); break;
+            default: m = rotate_unit_smem(xrow, c0, G, p.rnorm[a]); break;
           }
           amax = fmaxf(amax, m);
         }
