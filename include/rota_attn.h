@@ -54,7 +54,12 @@ typedef enum {
  *   that order at channel offsets 0, rope_dim[0], rope_dim[0]+rope_dim[1];
  *   each even, summing to head_dim (e.g. 44/42/42, 16/56/56, 16/24/24).
  * had_block: size of the Hadamard blocks of the rotation inside each
- *   partition: a power of two (1 = no rotation) dividing rope_dim[a], <= 64.
+ *   partition, dividing rope_dim[a], <= 64: a power of two (1 = no rotation;
+ *   Sylvester matrix, fast transform) or an order the library builds by
+ *   doubling (of an order >= 12), Paley I (n - 1 a prime = 3 mod 4) or
+ *   Paley II (n / 2 - 1 a prime = 1 mod 4), tried in that order -- 12, 20,
+ *   24, 28, 36, 40, 44, 48, 56, 60 -- applied as a dense product summed in
+ *   fp32 in column order.  Any other value is ROTA_ERR_INVALID_ARG.
  * rope_theta: RoPE base (10000).
  * sm_scale: softmax scale; 0 selects 1/sqrt(head_dim) (rounded to fp32).
  * rope_phase: per partition, an angle (radians, finite) added to every pair's
