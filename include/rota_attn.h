@@ -152,8 +152,9 @@ rota_status rota_attn_build_rope_tables(const rota_attn_desc* desc, float* host_
  *   head_flags      : host uint8 [H]; 1 = the head takes the FP16 fallback at this
  *                     call (per head, per denoising step), 0 = INT4.  NULL = all INT4.
  * INT4 heads: Q and K get RoPE (fp32, pair (2i, 2i+1) of each partition
- *   rotated by the table angle), then the normalised Sylvester Hadamard H_b/sqrt(b)
- *   on consecutive blocks of had_block[a] channels inside each partition, then
+ *   rotated by the table angle), then the normalised Hadamard matrix H_b/sqrt(b)
+ *   (Sylvester for a power of two, else the one described at had_block) on
+ *   consecutive blocks of had_block[a] channels inside each partition, then
  *   symmetric INT4 codes, one scale per 64 tokens x head_dim block:
  *   scale = amax/7, code = clamp(rne(y * (7/amax)), -7, 7).  V (no RoPE, no
  *   rotation) gets the same quantiser per channel per 64-token block.  Tokens
