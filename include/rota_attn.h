@@ -23,8 +23,11 @@
  *     with nothing enqueued.  Faults detected on the device (a bounded wait
  *     that ran out, a failed bounds check) are recorded in a device error
  *     word and reported by rota_attn_get_error.
- *   - Layouts are row-major with the last index fastest; s4 codes are packed
- *     two per byte, low nibble first, two's complement.
+ *   - Layouts are row-major with the last index fastest.  INT4 codes (values
+ *     in [-7, 7]) are sign-magnitude nibbles (bit 3 = sign, bits 0-2 =
+ *     magnitude), packed along the last axis in groups of 8 elements per
+ *     32-bit word: byte j of the word holds element j in its low nibble and
+ *     element j + 4 in its high nibble (j = 0..3).
  *   - Npad = 64 * ceil(N / 64); nblk = Npad / 64.
  */
 #ifndef ROTA_ATTN_H
