@@ -23,7 +23,10 @@
 // The exponentials use a reference max m_ref per row that is raised only when
 // a block's max exceeds it by more than 8 (log2 units): P stays <= 2^8, which
 // fp16 holds, and O and l are rescaled in place only then (a warp rescales
-// its TMEM rows after the previous P V has landed).  out = O / l.
+// its TMEM rows after the previous P V has landed).  The raise is voted per
+// warp and every row of the warp follows it; rows past N (whatever follows the
+// head in the Q view) take zero scores, so the vote depends on valid rows
+// only and the result does not depend on neighbouring memory.  out = O / l.
 #pragma once
 #include <cstdint>
 #include <cuda.h>

@@ -43,9 +43,10 @@
 //               running max, P codes (fp16) and their row sum, O rescale,
 //               epilogue out = O / l.
 // Per 64-key block j and tile t the MMA warp issues S_t(j) = Q_t K_j^T
-// (128 x 64, two TMEM buffers per tile so S_t(j+1) is computed while the
-// softmax works on block j) and, once tile t has written its P codes,
-// O_t += P_t V'_hi + P_t V'_lo (128 x D).
+// (128 x 64 into the tile's one S buffer in TMEM, which the softmax warps
+// release as soon as S is in their registers, so S_t(j+1) is computed while
+// they work on block j) and, once tile t has written its P codes into TMEM,
+// O_t += P_t V'_hi + P_t V'_lo (128 x D, O accumulated in TMEM).
 #pragma once
 #include <climits>
 #include <cstdint>
