@@ -316,6 +316,15 @@ rota_status rota_attn_fwd_int4_noalloc(const rota_attn_desc* desc, const uint16_
 /* ---------------------------------------------------------- test hooks --- */
 
 /*
+ * Host only: the Hadamard matrix the prologue uses for a block of the
+ * non-power-of-two order n (the construction described at had_block), as
+ * +1 / -1 into h (host int8 [n*n], row-major).  ROTA_ERR_UNSUPPORTED for an
+ * order it builds none of (powers of two included: those use the fast
+ * Sylvester transform), ROTA_ERR_INVALID_ARG for h NULL or n outside [2, 64].
+ */
+rota_status rota_attn_debug_hadamard(int32_t n, int8_t* h);
+
+/*
  * Runs the INT4 attention kernel for head (b, h) only, with its debug dump
  * enabled: for rows [r0, r0+nr) it also stores the s32 scores S (device int32
  * [nr, N]) and the P codes (device uint8 [nr, N]).  `out` as for

@@ -240,3 +240,16 @@ def test_validate_hadamard_orders(ra, had, ok):
 def test_validate_hunyuan_orders(ra, had):
     d = _desc(ra, synth.scaled(synth.WORKLOADS["hunyuan"], "v", had=had))
     assert ra.rota_attn_validate(d) == ra.ROTA_OK
+
+
+@pytest.mark.parametrize("n", range(2, 65))
+def test_library_hadamard_equals_oracle(ra, n):
+    """The library builds its non-power-of-two Hadamard matrices independently
+    of the oracle; bit-exact codes need the very same matrix for every order."""
+    st, h = ra.rota_attn_debug_hadamard(n)
+    ref = oracle.hadamard(n)
+    if ref is None:
+        assert st == ra.ROTA_ERR_UNSUPPORTED, n
+    else:
+        assert st == ra.ROTA_OK, n
+        assert np.array_equal(h, ref), n

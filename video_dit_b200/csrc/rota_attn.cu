@@ -731,6 +731,15 @@ rota_status rota_attn_debug_pcode(const float* dvals, uint8_t* u, int64_t n, voi
   return cuda_status(cudaGetLastError());
 }
 
+rota_status rota_attn_debug_hadamard(int32_t n, int8_t* h) {
+  if (!h || n < 2 || n > 64) return ROTA_ERR_INVALID_ARG;
+  uint64_t neg[64];
+  if (!hadamard_rows(n, neg)) return ROTA_ERR_UNSUPPORTED;
+  for (int i = 0; i < n; ++i)
+    for (int j = 0; j < n; ++j) h[i * n + j] = ((neg[i] >> j) & 1ull) ? -1 : 1;
+  return ROTA_OK;
+}
+
 rota_status rota_attn_debug_inject_timeout(int32_t arm, uint64_t timeout_ns) {
   std::lock_guard<std::mutex> g(g_inject.mu);
   g_inject.armed = arm ? 1 : 0;

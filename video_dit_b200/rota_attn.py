@@ -68,6 +68,7 @@ _SIGS = {
     "rota_attn_forward_host": ([_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _BUF, ctypes.c_int32, _P, _P],
                                ctypes.c_int),
     "rota_attn_head_error": ([_D, _P, _P, _P, _P], ctypes.c_int),
+    "rota_attn_debug_hadamard": ([ctypes.c_int32, _P], ctypes.c_int),
     "rota_attn_select_fp16_heads": ([_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_float, ctypes.c_int32, _P, _P],
                                     ctypes.c_int),
 }
@@ -204,6 +205,12 @@ def rota_attn_debug_dump_int4(desc, buffers, b, h, r0, nr, s_out, p_out, out, st
 
 def rota_attn_debug_pcode(d, u, stream=None) -> int:
     return _lib.rota_attn_debug_pcode(_ptr(d), _ptr(u), int(d.numel()), _stream(stream))
+
+
+def rota_attn_debug_hadamard(n: int):
+    """-> (status, int8 [n, n]): the library's Hadamard matrix of a non-power-of-two order."""
+    h = np.zeros((max(n, 1), max(n, 1)), np.int8)
+    return _lib.rota_attn_debug_hadamard(int(n), h.ctypes.data), h
 
 
 def rota_attn_debug_inject_timeout(arm: bool, timeout_ns: int = 0) -> int:
