@@ -134,8 +134,9 @@ def workload_config(w, l2_note):
 # DRAM bytes (read + write) per attention launch, from one ncu capture of the
 # current kernels on the F = 3 sweep point (B=1, H=40, N=4680, profiles/), per
 # (head, token): the traffic is the K/V images or tiles and the output, linear
-# in B * heads * N.  None = no capture of the current kernel version.
-TRAFFIC_PER_HEAD_TOKEN = {"attn_int4_kernel": 1035.70, "attn_fp16_kernel": 1076.75}
+# in B * heads * N.  A kernel missing here has no capture of its current
+# version, and its traffic is reported as null.
+TRAFFIC_PER_HEAD_TOKEN = {"attn_fp16_kernel": 1076.75}
 
 
 def traffic_per_launch(kernel, w, heads):
@@ -165,6 +166,30 @@ def oracle_sample(w, q, k, v, rows: int = 128):
                       f"of that head, {t2 - t0:.1f} s on 1 core, extrapolated linearly to "
                       f"B*H={w.B * w.H} heads x {w.N} rows",
             "seconds": t2 - t0}
+
+
+def accuracy_sample(w, q, k, v, out, h, rows):
+    """Accuracy of the GPU output on `rows` query rows (the middle ones) of
+    head h: max-abs error against the oracle's INT4 result, the largest error
+    relative to the row norm, and the cosine against unquantised attention
+    (RoPE, no rotation, no quantisation, double softmax)."""
+    import oracle
+    hs = (np.ascontiguousarray(x[:1, h:h + 1]) for x in (q, k, v))
+    qs, ks, vs = hs
+    sm = float(np.float32(1 / np.sqrt(w.d)))
+    r0 = max(0, w.N // 2 - rows // 2)
+    prep = oracle.prepare(qs, ks, vs, w.grid, w.rope_dim, w.had_block, w.theta, np.zeros(1, np.uint8),
+                          phase=w.rope_phase)
+    o4 = oracle.attn_int4(prep, w.N, sm, 0, 0, r0, rows)
+    unq = oracle.attn_ref(qs, ks, vs, w.grid, w.rope_dim, sm, 0, 0, r0, rows, theta=w.theta, phase=w.rope_phase)
+    got = out[0, h, r0:r0 + rows].double().cpu().numpy()
+    err = np.abs(got - o4)
+    rn = np.linalg.norm(o4, axis=-1)
+    cos = (got * unq).sum(-1) / (np.linalg.norm(got, axis=-1) * np.linalg.norm(unq, axis=-1) + 1e-30)
+    return {"head": h, "rows": f"{r0}..{r0 + rows - 1}", "max_abs_vs_oracle": float(err.max()),
+            "max_rel_row_norm": float((err.max(-1) / (rn + 1e-30)).max()),
+            "cos_vs_unquantised_mean": float(cos.mean()), "cos_vs_unquantised_min": float(cos.min()),
+            "tolerance_max_abs": 2e-3}
 
 
 def run_reference(args, w, world, rank):
@@ -208,6 +233,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024)     # the cpu_baseline sample (about 10 s)
     ap.add_argument("--chunk-heads", type=int, default=0)     # heads per chunk of the e2e pipeline (0: library default)
     ap.add_argument("--no-e2e", action="store_true")          # skip the end-to-end loop (profiling runs)
+    ap.add_argument("--accuracy-rows", type=int, default=32)  # sampled rows of the accuracy record (0: none)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -249,19 +275,23 @@ def main():
             pg.barrier()
 
     def step(ev=None):
-        # prologue, INT4 attention, FP16 fallback -- each kernel bracketed by events
+        # prologue, INT4 attention (its two launches: widening of the K / V
+        # codes, attention), FP16 fallback -- each kernel bracketed by events
         if ev is not None:
             ev[0].record(stream)
         att.prepare(qd, kd, vd, flags)
         if ev is not None:
             ev[1].record(stream)
-        ra._check(ra.rota_attn_fwd_int4(desc, att.buffers, flags, out), "fwd_int4")
+        ra._check(ra.rota_attn_int4_widen(desc, att.buffers, flags), "int4_widen")
         if ev is not None:
             ev[2].record(stream)
+        ra._check(ra.rota_attn_int4_attend(desc, att.buffers, flags, out), "int4_attend")
+        if ev is not None:
+            ev[3].record(stream)
         if any_fp16:
             ra._check(ra.rota_attn_fwd_fp16_fallback(desc, att.buffers, vd, flags, out), "fwd_fp16")
         if ev is not None:
-            ev[3].record(stream)
+            ev[4].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -273,7 +303,7 @@ def main():
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
@@ -286,8 +316,9 @@ def main():
     barrier()
     ms_total = t0.elapsed_time(t1)
     t_pro = [e[0].elapsed_time(e[1]) for e in evs]
-    t_int4 = [e[1].elapsed_time(e[2]) for e in evs]
-    t_f16 = [e[2].elapsed_time(e[3]) for e in evs]
+    t_widen = [e[1].elapsed_time(e[2]) for e in evs]
+    t_int4 = [e[2].elapsed_time(e[3]) for e in evs]
+    t_f16 = [e[3].elapsed_time(e[4]) for e in evs]
 
     ms_e2e, chunk_heads = 0.0, None
     if not args.no_e2e:
@@ -320,12 +351,14 @@ def main():
     if rank == 0:
         ops = w.ops()
         value = ops * world / (ms_step * 1e-3) / 1e12
-        # The timed region is K back-to-back steps (well over a second of
-        # tensor-core load on the large configs), so the denominators are the
-        # sustained (power-capped) measured peaks; the burst ones ride along.
-        int8_peak = peaks["bf16_sus"] * NOMINAL_INT8_PER_BF16
+        # The roofline kernel is timed per launch (its own CUDA events), so the
+        # denominators are the burst measured peaks; the sustained (power-
+        # capped, seconds-long loop) ones ride along.  INT8/FP8 dense = 2 x the
+        # measured bf16 GEMM (NVIDIA's nominal 4.5 : 2.25 ratio).
         int8_burst = peaks["bf16"] * NOMINAL_INT8_PER_BF16
+        int8_sus = peaks["bf16_sus"] * NOMINAL_INT8_PER_BF16
         ms_int4 = statistics.mean(t_int4)
+        ms_widen = statistics.mean(t_widen)
         ms_f16 = statistics.mean(t_f16)
         ms_pro = statistics.mean(t_pro)
         n_int4_heads = int((flags == 0).sum())
@@ -333,19 +366,19 @@ def main():
         ops_f16 = 4.0 * w.B * int(flags.sum()) * w.N * w.N * w.d
         if ms_int4 >= ms_f16:
             kern, achieved = "attn_int4_kernel", (ops_int4 / (ms_int4 * 1e-3) / 1e12 if n_int4_heads else 0.0)
-            rl = {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": int8_peak,
-                  "unit": "TOPS (INT8 dense)", "frac": achieved / int8_peak,
-                  "peak_source": f"{peaks['source']} bf16 sustained {peaks['bf16_sus']} TFLOP/s x nominal INT8/BF16 "
-                                 f"ratio 2 (burst: {int8_burst:.1f}, frac {achieved / int8_burst:.3f})",
+            rl = {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": int8_burst,
+                  "unit": "TOPS (INT8 dense)", "frac": achieved / int8_burst,
+                  "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} TFLOP/s x nominal INT8/BF16 "
+                                 f"ratio 2 (of measured; sustained: {int8_sus:.1f}, frac {achieved / int8_sus:.3f})",
                   "traffic": traffic_per_launch(kern, w, n_int4_heads), "algorithmic_ops_per_launch": ops_int4,
                   "int8_spec_frac": achieved / INT8_SPEC_TOPS}
         else:
             kern = "attn_fp16_kernel"
             achieved = ops_f16 / (ms_f16 * 1e-3) / 1e12
-            rl = {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sus"],
-                  "unit": "TFLOP/s (FP16/BF16 dense)", "frac": achieved / peaks["bf16_sus"],
-                  "peak_source": f"{peaks['source']} bf16 sustained {peaks['bf16_sus']} TFLOP/s "
-                                 f"(burst: {peaks['bf16']}, frac {achieved / peaks['bf16']:.3f})",
+            rl = {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16"],
+                  "unit": "TFLOP/s (FP16/BF16 dense)", "frac": achieved / peaks["bf16"],
+                  "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} TFLOP/s (of measured; "
+                                 f"sustained: {peaks['bf16_sus']}, frac {achieved / peaks['bf16_sus']:.3f})",
                   "traffic": traffic_per_launch(kern, w, int(flags.sum())), "algorithmic_ops_per_launch": ops_f16}
         # prologue algorithmic bytes: fp16 Q,K,V read; packed codes + scales written
         nblk = (w.N + 63) // 64
@@ -360,7 +393,8 @@ def main():
             "config": workload_config(w, "inputs > L2: fp16 Q/K/V %.2f GB, INT4 codes %.2f GB per step, no flush"
                                       % (3 * q.nbytes / 1e9, 3 * w.B * w.H * nblk * 64 * w.d / 2 / 1e9)),
             "pct_int8_spec": 100.0 * value / world / INT8_SPEC_TOPS,
-            "breakdown_ms": {"prologue": ms_pro, "int4_attention": ms_int4, "fp16_fallback": ms_f16},
+            "breakdown_ms": {"prologue": ms_pro, "int4_widen": ms_widen, "int4_attention": ms_int4,
+                             "fp16_fallback": ms_f16},
             "prologue_gbs": pro_bytes / (ms_pro * 1e-3) / 1e9,
             "roofline": rl,
             "e2e": None if args.no_e2e else {
@@ -370,6 +404,9 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }
+        if args.accuracy_rows > 0 and n_int4_heads:
+            h_acc = int(np.flatnonzero(flags == 0)[min(17, n_int4_heads - 1)])
+            line["accuracy"] = accuracy_sample(w, q, k, v, out, h_acc, args.accuracy_rows)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = oracle_sample(w, q, k, v, rows=args.cpu_rows)
             line["cpu_baseline"].pop("seconds", None)

@@ -95,13 +95,12 @@ typedef struct {
  *   rope_cos, rope_sin: fp32 tables from rota_attn_build_rope_tables, copied
  *                      to the device by the caller.
  *   int4_work        : workspace of rota_attn_fwd_int4 (bytes[ROTA_BUF_INT4_WORK],
- *                      320 * head_dim bytes per (head, 64-key block)): the K
- *                      and V codes of the INT4 heads widened once per call into
- *                      pre-swizzled tensor-core operand images -- K as e4m3
- *                      (64 x head_dim), V with its channel scale folded in as
- *                      two exact fp16 tiles v * s_hi and v * s_lo (head_dim x 64
- *                      each).  Transient: its contents are rewritten by every
- *                      call.
+ *                      64 * head_dim + 8192 bytes per (head, 64-key block)): the
+ *                      K and V codes of the INT4 heads widened once per call
+ *                      into pre-swizzled tensor-core operand images of exact
+ *                      e4m3 values -- K as 64 x head_dim, V transposed as 128
+ *                      channel rows x 64 keys (rows past head_dim zero).
+ *                      Transient: its contents are rewritten by every call.
  */
 typedef struct {
   uint8_t* q_codes;
@@ -170,19 +169,35 @@ rota_status rota_attn_prepare_qk(const rota_attn_desc* desc, const uint16_t* q, 
 
 /*
  * INT4 attention (the abstract's mixed-precision INT4 FlashAttention) for the
- * heads whose flag is 0.  Integer Q K^T on the tensor cores (s32); scores
+ * heads whose flag is 0.  Exact integer Q K^T on the tensor cores (the codes
+ * as exact e4m3 values, fp32 accumulation that stays integral); scores
  * dequantised with c = (sq * sk) * (sm_scale * log2 e); a running max m over
  * consecutive 64-key groups; range-optimised P codes u = rne(15 * 2^(S c - m))
  * in 0..15 (fixed scale 1/15, zero-point 0: the whole unsigned 4-bit range,
- * as the abstract's "Range-optimized P Quantization" asks); integer P V on
- * the tensor cores per 64-key block; V scales, rescaling by 2^(m_old - m_new)
- * and the row sum of the codes in fp32; out = O / l.  Two launches: the K / V
- * codes are first widened once into buf->int4_work, then the attention kernel
- * streams the widened tiles with TMA bulk copies.
+ * as the abstract's "Range-optimized P Quantization" asks); exact integer
+ * P V per 64-key block on the tensor cores, the same way; then, in fp32 on
+ * the CUDA cores, each block's per-channel V scales, the rescaling of O by
+ * 2^(m_old - m_new) where a row's max moved, and the row sum of the codes;
+ * out = O / l.  Two launches: the K / V codes are first widened once into
+ * buf->int4_work, then the attention kernel streams the widened tiles with
+ * bulk copies.
  *   out: fp32 [B,H,N,head_dim]; rows of flagged heads are not written.
  */
 rota_status rota_attn_fwd_int4(const rota_attn_desc* desc, const rota_attn_buffers* buf,
                                const uint8_t* head_flags, float* out, void* stream);
+
+/*
+ * The two launches of rota_attn_fwd_int4 as separate calls (same arguments;
+ * rota_attn_fwd_int4 == rota_attn_int4_widen then rota_attn_int4_attend on
+ * the same stream), so that each kernel can be timed on its own:
+ * rota_attn_int4_widen writes buf->int4_work from the K / V codes of the
+ * INT4 heads; rota_attn_int4_attend reads it and writes out.  The attend call
+ * must follow a widen call on the same codes and flags.
+ */
+rota_status rota_attn_int4_widen(const rota_attn_desc* desc, const rota_attn_buffers* buf,
+                                 const uint8_t* head_flags, void* stream);
+rota_status rota_attn_int4_attend(const rota_attn_desc* desc, const rota_attn_buffers* buf,
+                                  const uint8_t* head_flags, float* out, void* stream);
 
 /*
  * FP16 fallback (the abstract's "selective FP16 fallback") for the heads whose
@@ -293,14 +308,16 @@ const char* rota_attn_status_string(rota_status s);
  * every head takes the INT4 path (no FP16 fallback).  The intermediate codes,
  * scales and RoPE tables live in one 16 MiB array in the library's static
  * device memory, which every GPU that loads the library holds until exit.
- * Its size bounds the problem: B*H*nblk*(420*head_dim + 8) bytes of codes,
+ * Its size bounds the problem: B*H*nblk*(164*head_dim + 8200) bytes of codes,
  * widened tiles and scales plus the RoPE tables (each entry padded to 256 bytes)
  * must fit in ROTA_NOALLOC_SCRATCH_BYTES, and each RoPE table in
  * ROTA_NOALLOC_MAX_TABLE floats; larger problems return
  * ROTA_ERR_UNSUPPORTED, with nothing enqueued.
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  The RoPE tables are copied from a static host
+ * (cudaGetSymbolAddress) with that device current and keeps it; make that
+ * first call before any stream capture.  A device reset (cudaDeviceReset)
+ * invalidates the kept address: after one, do not call this entry point
+ * again in the same process.  The RoPE tables are copied from a static host
  * buffer with a pageable cudaMemcpyAsync, which synchronises `stream` first.
  * All calls share the one array and it keeps the last call's contents (every
  * byte a call reads is written earlier in the same call, so nothing has to

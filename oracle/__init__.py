@@ -71,7 +71,7 @@ def lib():
         L.oracle_pcode.restype = i32
         L.oracle_pcode_array.argtypes = [P, P, i64, P]
         L.oracle_pcode_array.restype = None
-        L.oracle_attn_int4.argtypes = [i32, i32, i32, i32, f32, i32] + [P] * 6 + \
+        L.oracle_attn_int4.argtypes = [i32, i32, i32, i32, f32, i32, i32] + [P] * 6 + \
             [i32, i32, i32, i32, i32, P, P, P]
         L.oracle_attn_int4.restype = i32
         L.oracle_attn_fp16.argtypes = [i32, i32, i32, i32, f32, P, P, P, i32, i32, i32, i32, P]
@@ -221,16 +221,18 @@ def prepare(q, k, v, grid, rope_dim, had_block, theta=10000.0, flags=None, phase
 
 
 def attn_int4(prep: dict, N: int, sm_scale: float, b: int, h: int, r0: int, nr: int,
-              group: int = 64, online: bool = False, dump: bool = False):
+              group: int = 64, online: bool = False, dump: bool = False, rowsum: int = 0):
     """INT4 attention rows [r0, r0+nr) of head (b,h).  Returns out [nr,d] (double)
-    and, if dump, S_int [nr,N] int32 and P codes [nr,N] uint8."""
+    and, if dump, S_int [nr,N] int32 and P codes [nr,N] uint8.  group: key group
+    of the running max (64 or 128); rowsum: 0 = sum of the codes (R2), 1 = sum
+    of the unquantised 15 * 2^d (R1)."""
     qc = prep["q_codes"]
     B, H, _, dh = qc.shape
     d = dh * 2
     out = np.zeros((nr, d), np.float64)
     s = np.zeros((nr, N), np.int32) if dump else None
     p = np.zeros((nr, N), np.uint8) if dump else None
-    bad = lib().oracle_attn_int4(B, H, N, d, float(sm_scale), int(group),
+    bad = lib().oracle_attn_int4(B, H, N, d, float(sm_scale), int(group), int(rowsum),
                                  _p(qc), _p(prep["k_codes"]), _p(prep["q_scale"]),
                                  _p(prep["k_scale"]), _p(prep["v_codes"]), _p(prep["v_scale"]),
                                  b, h, r0, nr, int(online),

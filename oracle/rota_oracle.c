@@ -163,8 +163,8 @@ static void rope_row(const float *x, float *y, long n, const int grid[3], const 
 /* Q K^T is unchanged in exact arithmetic; V is not rotated.               */
 /* ----------------------------------------------------------------------- */
 
-/* Blocks whose size is not a power of two (the survey's numerics variant:  */
-/* the partition's own size, e.g. 44 for a 44-channel partition) take a     */
+/* Blocks whose size is not a power of two (a numerics option: e.g. the    */
+/* partition's own size, 44 for a 44-channel partition) take a            */
 /* Hadamard matrix of that order from the classical constructions:          */
 /*   Paley I  (q prime, q = 3 mod 4), order q + 1:  H = I + S,             */
 /*            S = [[0, 1^T], [-1, Q]],  Q_ij = chi(j - i);                  */
@@ -506,14 +506,21 @@ void oracle_pcode_array(const float *d, uint8_t *u, long n, int *bad)
 /*  out[c]     = sum_g 2^(m_g - M) sv[g,c] sum_{k in g} u_k vcode[k,c]      */
 /*               / sum_g 2^(m_g - M) sum_{k in g} u_k        (double)       */
 /* The row sum uses the quantised P, the same values that multiply V        */
-/* (reading); the 1/15 scale cancels.  `online` selects the recurrence form */
+/* (reading R2, rowsum = 0); the 1/15 scale cancels.  rowsum = 1 takes the  */
+/* other reading of the page's row sum, the unquantised P (R1):            */
+/*  out[c]     = sum_g 2^(m_g - M) sv[g,c] sum_{k in g} u_k vcode[k,c]      */
+/*               / sum_g 2^(m_g - M) sum_{k in g} 15 * 2^(d_k)  (double)    */
+/* with d_k the same fp32 exponent the code u_k is taken from (15 P_k      */
+/* unrounded, so P = u / 15 in the numerator).  `group` is the key group   */
+/* of the running max (64 = the quant block; 128 spans two blocks, whose    */
+/* codes then share one max).  `online` selects the recurrence form */
 /* O <- O 2^(m_{g-1}-m_g) + ..., l <- l 2^(m_{g-1}-m_g) + ... instead of the */
 /* closed form; both are kept so they can be checked against each other.    */
 /* s_dump [nr,N] and p_dump [nr,N] may be NULL.  Returns the number of      */
 /* margin violations in the P codes (0 expected).                          */
 /* ----------------------------------------------------------------------- */
 
-int oracle_attn_int4(int B, int H, int N, int d, float sm_scale, int group,
+int oracle_attn_int4(int B, int H, int N, int d, float sm_scale, int group, int rowsum,
                      const uint8_t *q_codes, const uint8_t *k_codes, const float *q_scale,
                      const float *k_scale, const uint8_t *v_codes, const float *v_scale,
                      int b, int h, int r0, int nr, int online,
@@ -540,7 +547,8 @@ int oracle_attn_int4(int B, int H, int N, int d, float sm_scale, int group,
     float *mg = (float *)malloc(sizeof(float) * (size_t)ngroup);
     int *qrow = (int *)malloc(sizeof(int) * (size_t)d);
     double *num = (double *)malloc(sizeof(double) * (size_t)d);
-    if (!S || !cs || !U || !mg || !qrow || !num) return -1;
+    double *rs = (double *)malloc(sizeof(double) * (size_t)N);   /* row-sum weight of each key */
+    if (!S || !cs || !U || !mg || !qrow || !num || !rs) return -1;
 
     for (int i = r0; i < r0 + nr; ++i) {
         for (int c = 0; c < d; ++c) qrow[c] = code_at(qc + (long)i * (d / 2), c);
@@ -566,13 +574,15 @@ int oracle_attn_int4(int B, int H, int N, int d, float sm_scale, int group,
         for (long kk = 0; kk < N; ++kk) {
             float dd = fmaf((float)S[kk], cs[kk], -mg[kk / group]);
             U[kk] = (uint8_t)oracle_pcode(dd, &bad);
+            rs[kk] = rowsum ? 15.0 * exp2((double)dd) : (double)U[kk];
         }
         double den = 0.0;
         for (int c = 0; c < d; ++c) num[c] = 0.0;
         if (!online) {
             for (long kk = 0; kk < N; ++kk) {
-                double w = exp2((double)mg[kk / group] - (double)M) * (double)U[kk];
-                den += w;
+                double wg = exp2((double)mg[kk / group] - (double)M);
+                double w = wg * (double)U[kk];
+                den += wg * rs[kk];
                 if (U[kk] == 0) continue;
                 long j = kk / QB, t = kk % QB;
                 for (int c = 0; c < d; ++c) {
@@ -587,7 +597,7 @@ int oracle_attn_int4(int B, int H, int N, int d, float sm_scale, int group,
                 den *= alpha;
                 for (int c = 0; c < d; ++c) num[c] *= alpha;
                 for (long kk = (long)g * group; kk < N && kk < (long)(g + 1) * group; ++kk) {
-                    den += (double)U[kk];
+                    den += rs[kk];
                     long j = kk / QB, t = kk % QB;
                     for (int c = 0; c < d; ++c) {
                         int vcode = code_at(vc + (j * d + c) * 32, t);
@@ -601,7 +611,7 @@ int oracle_attn_int4(int B, int H, int N, int d, float sm_scale, int group,
         if (s_dump) memcpy(s_dump + (long)(i - r0) * N, S, sizeof(int32_t) * (size_t)N);
         if (p_dump) memcpy(p_dump + (long)(i - r0) * N, U, (size_t)N);
     }
-    free(S); free(cs); free(U); free(mg); free(qrow); free(num);
+    free(S); free(cs); free(U); free(mg); free(qrow); free(num); free(rs);
     return bad;
 }
 

@@ -28,3 +28,21 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Accuracy of the INT4 path on the GPU parity cases: max-abs error against
+    the oracle, error relative to the row norm, cosine against unquantised
+    attention."""
+    try:
+        import gpu_util
+    except Exception:
+        return
+    if not gpu_util.ACCURACY:
+        return
+    terminalreporter.write_sep("-", "INT4 accuracy (vs oracle; cosine vs unquantised attention)")
+    for name, r in gpu_util.ACCURACY:
+        terminalreporter.write_line(
+            f"{name:40s} max_abs {r['max_abs_vs_oracle']:.3e}  rel_row_norm {r['max_rel_row_norm']:.3e}  "
+            f"cos_unq mean {r['cos_vs_unquantised_mean']:.4f} min {r['cos_vs_unquantised_min']:.4f}  "
+            f"rows {r['rows']}")

@@ -49,6 +49,12 @@ def run(w: synth.Workload, q, k, v, flags=None, dump=None):
     return codes, out.cpu().numpy(), dumped
 
 
+def kappa(head_dim: int) -> float:
+    """The score scale's constant both sides use: RN(RN(1/sqrt(d)) * log2 e) from double."""
+    s = np.float32(1.0 / math.sqrt(head_dim))
+    return float(np.float32(np.float64(s) * 1.4426950408889634))
+
+
 def sm_scale(w):
     return float(np.float32(1 / math.sqrt(w.d)))
 
@@ -59,3 +65,30 @@ def row_stats(got, ref):
     rn = np.linalg.norm(ref, axis=-1, keepdims=True)
     cos = (got * ref).sum(-1) / (np.linalg.norm(got, axis=-1) * rn[..., 0] + 1e-30)
     return float(err.max()), float((err / (rn + 1e-30)).max()), float(cos.min())
+
+
+# Accuracy records of this session's parity tests, printed at the end of the
+# run (conftest.pytest_terminal_summary).
+ACCURACY = []
+
+
+def accuracy(w: synth.Workload, q, k, v, got, o_int4, b, h, r0, nr):
+    """The accuracy record of rows [r0, r0+nr) of head (b, h): max-abs error
+    against the oracle's INT4 result, the largest error relative to the row
+    norm, and the cosine of the output against unquantised attention (RoPE,
+    no rotation, no quantisation, double softmax; oracle.attn_ref)."""
+    import oracle
+    unq = oracle.attn_ref(q, k, v, w.grid, w.rope_dim, sm_scale(w), b, h, r0, nr, theta=w.theta,
+                          phase=w.rope_phase)
+    err = np.abs(got - o_int4)
+    rn = np.linalg.norm(o_int4, axis=-1)
+    cos = (got * unq).sum(-1) / (np.linalg.norm(got, axis=-1) * np.linalg.norm(unq, axis=-1) + 1e-30)
+    return {"max_abs_vs_oracle": float(err.max()),
+            "max_rel_row_norm": float((err.max(-1) / (rn + 1e-30)).max()),
+            "cos_vs_unquantised_mean": float(cos.mean()), "cos_vs_unquantised_min": float(cos.min()),
+            "rows": int(nr)}
+
+
+def report(name: str, rec: dict):
+    ACCURACY.append((name, rec))
+    return rec

@@ -104,13 +104,6 @@ def test_rope_tables_identical_to_oracle(ra, name):
     assert np.array_equal(s.view(np.uint32), os_.view(np.uint32))
 
 
-def test_kappa_matches_oracle_definition(ra):
-    # the oracle's kappa: RN(RN(1/sqrt(d)) * log2 e) from double
-    for d in (64, 128):
-        sm = np.float32(1 / np.sqrt(d))
-        assert ra.kappa(d) == np.float32(np.float64(sm) * 1.4426950408889634074)
-
-
 # ----------------------------------------------- host-to-host pipeline (host logic)
 
 @pytest.mark.parametrize("name", ["wan480", "wan720", "hunyuan"])

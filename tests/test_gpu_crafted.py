@@ -19,6 +19,7 @@ import oracle
 from video_dit_b200 import synth
 
 from gpu_util import desc_of, lib, row_stats
+from gpu_util import kappa as gpu_kappa
 
 TOL = 2e-3
 pytestmark = pytest.mark.gpu
@@ -70,7 +71,7 @@ def test_near_threshold_codes_rescales_and_exact_tie():
     assert w.N == N
     desc = desc_of(w)
     sm = float(np.float32(1 / math.sqrt(d)))
-    kappa = np.float32(ra.kappa(d))
+    kappa = np.float32(gpu_kappa(d))
     rng = np.random.default_rng(11)
 
     # Q: channel 0 only, 1 on even rows and 2 on odd rows.  K: channel 0 carries

@@ -12,7 +12,7 @@ import pytest
 import oracle
 from video_dit_b200 import synth
 
-from gpu_util import row_stats, run, sm_scale
+from gpu_util import accuracy, report, row_stats, run, sm_scale
 
 pytestmark = pytest.mark.gpu
 
@@ -69,6 +69,7 @@ def test_int4_scores_and_pcodes_bit_exact(name):
     assert np.array_equal(s, s_ref)
     assert np.array_equal(p, p_ref)
     e, rel, cos = row_stats(out[0, h, r0:r0 + nr], o_ref)
+    report(f"parity/{name} h{h}", accuracy(w, q, k, v, out[0, h, r0:r0 + nr], o_ref, 0, h, r0, nr))
     assert e <= TOL, (e, rel, cos)
 
 
@@ -146,6 +147,7 @@ def test_int4_long_sequence_sampled_rows():
     assert np.array_equal(s, s_ref)
     assert np.array_equal(p, p_ref)
     e, rel, cos = row_stats(out[0, h, r0:r0 + nr], o_ref)
+    report(f"parity/long h{h}", accuracy(w, q, k, v, out[0, h, r0:r0 + nr], o_ref, 0, h, r0, nr))
     assert e <= TOL, (e, rel, cos)
     o0 = oracle.attn_int4(ref, w.N, sm_scale(w), 0, 0, 0, 64)          # first rows of the other head
     assert row_stats(out[0, 0, :64], o0)[0] <= TOL

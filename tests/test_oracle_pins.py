@@ -104,6 +104,61 @@ def test_rope_row_matches_transformers_apply():
             off += d_a
 
 
+@pytest.mark.parametrize("rope_dim,grid", [((44, 42, 42), (21, 30, 52)), ((16, 56, 56), (33, 34, 60)),
+                                           ((16, 24, 24), (4, 8, 8))])
+def test_rope_rounding_order_bit_exact(rope_dim, grid):
+    """The RoPE arithmetic defines the quantiser's inputs bit for bit: pair
+    (2i, 2i+1) of partition a at position p becomes
+    y0 = RN(RN(x0 c) - RN(x1 s)), y1 = RN(RN(x0 s) + RN(x1 c)), every product
+    and sum a separate fp32 rounding (no fused multiply-add), c / s the fp32
+    table entries.  numpy float32 scalars round each operation once, in the
+    order written here, so a contracted FMA or a swapped operand in the oracle
+    changes some of these bits."""
+    c_tab, s_tab = oracle.rope_tables(grid, rope_dim)
+    rng = np.random.default_rng(11)
+    d = sum(rope_dim)
+    T, Hh, W = grid
+    toks = [0, 1, W, Hh * W, T * Hh * W - 1] + list(rng.integers(0, T * Hh * W, 40))
+    halves = [r // 2 for r in rope_dim]
+    toff = [0, T * halves[0], T * halves[0] + Hh * halves[1]]
+    for n in toks:
+        n = int(n)
+        pos = (n // (Hh * W), (n // W) % Hh, n % W)
+        x = (rng.standard_normal(d) * rng.choice([1.0, 15.0, 300.0], d)).astype(np.float32)
+        got = oracle.rope_rotate_row(x, n, grid, rope_dim, (1, 1, 1), rotate=False)
+        want = np.empty(d, np.float32)
+        off = 0
+        for a in range(3):
+            for i in range(halves[a]):
+                c = np.float32(c_tab[toff[a] + pos[a] * halves[a] + i])
+                s_ = np.float32(s_tab[toff[a] + pos[a] * halves[a] + i])
+                x0, x1 = np.float32(x[off + 2 * i]), np.float32(x[off + 2 * i + 1])
+                want[off + 2 * i] = np.float32(np.float32(x0 * c) - np.float32(x1 * s_))
+                want[off + 2 * i + 1] = np.float32(np.float32(x0 * s_) + np.float32(x1 * c))
+            off += rope_dim[a]
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32)), n
+
+
+def test_unquantised_reference_matches_torch_sdpa_float64():
+    """oracle.attn_ref (the reference of the cosine report): fp32 RoPE rows,
+    no rotation, no rounding to fp16, softmax attention in double; against
+    torch's float64 scaled_dot_product_attention on the same RoPE'd rows."""
+    w = synth.scaled(synth.WORKLOADS["wan480"], "ref_pin", H=2, grid=(2, 5, 9))      # N = 90
+    q, k, v = synth.make_inputs(w, seed=4)
+    sm = float(np.float32(1 / math.sqrt(w.d)))
+    for h in range(w.H):
+        qr = np.stack([oracle.rope_rotate_row(q[0, h, n].astype(np.float32), n, w.grid, w.rope_dim,
+                                              w.had_block, rotate=False) for n in range(w.N)])
+        kr = np.stack([oracle.rope_rotate_row(k[0, h, n].astype(np.float32), n, w.grid, w.rope_dim,
+                                              w.had_block, rotate=False) for n in range(w.N)])
+        vv = v[0, h].astype(np.float64)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(qr.astype(np.float64))[None], torch.from_numpy(kr.astype(np.float64))[None],
+            torch.from_numpy(vv)[None], scale=sm)[0].numpy()
+        got = oracle.attn_ref(q, k, v, w.grid, w.rope_dim, sm, 0, h, 0, w.N)
+        assert np.abs(got - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+
+
 def test_rope_identity_at_origin_and_relative_position():
     rope_dim, grid = (16, 24, 24), (4, 8, 8)
     rng = np.random.default_rng(2)
@@ -487,3 +542,87 @@ def test_int4_close_to_unquantised_attention_on_plain_gaussians():
     ref = oracle.attn_ref(q, k, v, w.grid, w.rope_dim, 1 / math.sqrt(w.d), 0, 0, 0, w.N)
     cos = (out * ref).sum(1) / np.linalg.norm(out, axis=1) / np.linalg.norm(ref, axis=1)
     assert cos.mean() > 0.93 and cos.min() > 0.75
+
+
+# ------------------------------------------------- numerics options (R1, G = 128)
+
+def _unit_c_scales(sm_scale):
+    """(sq, sk) with c = RN(RN(sq sk) kappa) == 1 exactly, kappa = RN(sm_scale log2 e)."""
+    kappa = np.float32(np.float64(np.float32(sm_scale)) * 1.4426950408889634074)
+    base = np.float32(1.0) / kappa
+    for step in range(-64, 65):
+        sk = np.array([base], np.float32).view(np.int32).__add__(np.int32(step)).view(np.float32)[0]
+        if np.float32(np.float32(np.float32(1.0) * sk) * kappa) == np.float32(1.0):
+            return np.float32(1.0), sk
+    raise AssertionError("no key scale gives c = 1")
+
+
+def _hand_prep(q_rows, k_rows, v_blocks, sq, sk, d=8):
+    """A one-head prepared problem from explicit codes: q_rows [n, d], k_rows
+    [N, d] (codes in [-7, 7]), v_blocks [nblk, d, 64]; every scale is 1 except
+    the Q / K block scales sq, sk."""
+    N = len(k_rows)
+    nblk = (N + 63) // 64
+    npad = nblk * 64
+    q = np.zeros((npad, d), np.int32)
+    q[:len(q_rows)] = q_rows
+    k = np.zeros((npad, d), np.int32)
+    k[:N] = k_rows
+    return {"q_codes": oracle.pack_codes(q)[None, None], "k_codes": oracle.pack_codes(k)[None, None],
+            "q_scale": np.full((1, 1, nblk), sq, np.float32), "k_scale": np.full((1, 1, nblk), sk, np.float32),
+            "v_codes": oracle.pack_codes(np.asarray(v_blocks, np.int32))[None, None],
+            "v_scale": np.ones((1, 1, nblk, d), np.float32)}
+
+
+def test_row_sum_readings_closed_form():
+    """Two keys with scores x = 1 and x = 0 (c = 1): exponents d = 0 and -1,
+    codes 15 and 8 (7.5 rounds to even), unquantised 15 * 2^d = 15 and 7.5.
+    R2 divides by the code sum 23, R1 by 22.5; the numerator is
+    15 v0 + 8 v1 either way."""
+    sm = 0.125
+    sq, sk = _unit_c_scales(sm)
+    qr = np.zeros((1, 8), np.int32)
+    qr[0, 0] = 1
+    kr = np.zeros((2, 8), np.int32)
+    kr[0, 0] = 1                                   # S = 1 -> x = 1 = the max
+    vb = np.zeros((1, 8, 64), np.int32)
+    vb[0, :, 0] = [1, -2, 3, -4, 5, -6, 7, 0]      # key 0
+    vb[0, :, 1] = [7, 6, 5, 4, 3, 2, 1, -1]        # key 1
+    prep = _hand_prep(qr, kr, vb, sq, sk)
+    o2, s, u = oracle.attn_int4(prep, 2, sm, 0, 0, 0, 1, dump=True)
+    o1 = oracle.attn_int4(prep, 2, sm, 0, 0, 0, 1, rowsum=1)
+    assert s.tolist() == [[1, 0]] and u.tolist() == [[15, 8]]
+    num = 15.0 * vb[0, :, 0] + 8.0 * vb[0, :, 1]
+    assert np.abs(o2[0] - num / 23.0).max() < 1e-15
+    assert np.abs(o1[0] - num / 22.5).max() < 1e-15
+
+
+def test_max_group_128_closed_form():
+    """Block 0: 64 keys with x = 0; block 1: key 64 with x = 1, the other 63
+    with x = 0 (c = 1).  With 64-key groups block 0 is coded against its own
+    max 0 (codes 15, weight 2^(0 - 1) = 1/2 at the end); with 128-key groups
+    both blocks share the max 1 (block 0's codes drop to 8, weight 1).  V codes
+    are 1 in block 0 and 2 in block 1 (all channels), every scale 1."""
+    sm = 0.125
+    sq, sk = _unit_c_scales(sm)
+    qr = np.zeros((1, 8), np.int32)
+    qr[0, 0] = 1
+    kr = np.zeros((128, 8), np.int32)
+    kr[64, 0] = 1
+    vb = np.zeros((2, 8, 64), np.int32)
+    vb[0] = 1
+    vb[1] = 2
+    prep = _hand_prep(qr, kr, vb, sq, sk)
+    o64, _, u64 = oracle.attn_int4(prep, 128, sm, 0, 0, 0, 1, group=64, dump=True)
+    o128, _, u128 = oracle.attn_int4(prep, 128, sm, 0, 0, 0, 1, group=128, dump=True)
+    assert (u64[0, :64] == 15).all() and u64[0, 64] == 15 and (u64[0, 65:] == 8).all()
+    assert (u128[0, :64] == 8).all() and u128[0, 64] == 15 and (u128[0, 65:] == 8).all()
+    num64 = 0.5 * 64 * 15 * 1 + (15 + 63 * 8) * 2
+    den64 = 0.5 * 64 * 15 + (15 + 63 * 8)
+    num128 = 64 * 8 * 1 + (15 + 63 * 8) * 2
+    den128 = 64 * 8 + (15 + 63 * 8)
+    assert np.abs(o64[0] - num64 / den64).max() < 1e-14
+    assert np.abs(o128[0] - num128 / den128).max() < 1e-14
+    # R1 with 128-key groups: 15 * 2^-1 = 7.5 per block-0 key and per other block-1 key
+    o128r1 = oracle.attn_int4(prep, 128, sm, 0, 0, 0, 1, group=128, rowsum=1)
+    assert np.abs(o128r1[0] - num128 / (64 * 7.5 + 15 + 63 * 7.5)).max() < 1e-14

@@ -377,12 +377,13 @@ rota_status rota_attn_prepare_qk(const rota_attn_desc* d, const uint16_t* q, con
   return cuda_status(cudaGetLastError());
 }
 
+// part: 1 = widen only, 2 = attention only, 3 = both
 static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers* buf, const uint8_t* head_flags,
                                float* out, void* stream, bool dump, int b, int h, int r0, int nr, int32_t* s_out,
-                               uint8_t* p_out) {
+                               uint8_t* p_out, int part = 3) {
   rota_status st = rota_attn_validate(d);
   if (st != ROTA_OK) return st;
-  if (!buf || !out || !aligned16(out)) return ROTA_ERR_INVALID_ARG;
+  if (!buf || ((part & 2) && (!out || !aligned16(out)))) return ROTA_ERR_INVALID_ARG;
   if (!int4_buffers_ok(buf, true)) return ROTA_ERR_INVALID_ARG;
 
   static rota::Int4Params p;  // large (heads list); filled under a lock below
@@ -436,26 +437,38 @@ static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers*
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // 1. widen the K / V codes of the selected heads once
-  const dim3 wgrid(p.nblk, p.nheads, batches);
-  if (d->head_dim == 128)
-    rota::widen_kv_kernel<128><<<wgrid, 256, 0, s>>>(p, const_cast<uint8_t*>(p.work));
-  else
-    rota::widen_kv_kernel<64><<<wgrid, 256, 0, s>>>(p, const_cast<uint8_t*>(p.work));
-  if ((st = cuda_status(cudaGetLastError())) != ROTA_OK) return st;
+  if (part & 1) {
+    const dim3 wgrid(p.nblk, p.nheads, batches);
+    if (d->head_dim == 128)
+      rota::widen_kv_kernel<128><<<wgrid, 256, 0, s>>>(p, const_cast<uint8_t*>(p.work));
+    else
+      rota::widen_kv_kernel<64><<<wgrid, 256, 0, s>>>(p, const_cast<uint8_t*>(p.work));
+    if ((st = cuda_status(cudaGetLastError())) != ROTA_OK) return st;
+  }
+  if (!(part & 2)) return ROTA_OK;
   // 2. attention
   const dim3 grid((d->N + rota::kRowsPerCta - 1) / rota::kRowsPerCta, p.nheads, batches);
+  // the debug dump runs the same kernel with its dump pointers set
   if (d->head_dim == 128)
-    st = dump ? launch_int4_kernel(rota::attn_int4_kernel<128, true>, rota::Int4Smem<128>::ALLOC, grid, s, p)
-              : launch_int4_kernel(rota::attn_int4_kernel<128, false>, rota::Int4Smem<128>::ALLOC, grid, s, p);
+    st = launch_int4_kernel(rota::attn_int4_kernel<128>, rota::Int4Smem<128>::ALLOC, grid, s, p);
   else
-    st = dump ? launch_int4_kernel(rota::attn_int4_kernel<64, true>, rota::Int4Smem<64>::ALLOC, grid, s, p)
-              : launch_int4_kernel(rota::attn_int4_kernel<64, false>, rota::Int4Smem<64>::ALLOC, grid, s, p);
+    st = launch_int4_kernel(rota::attn_int4_kernel<64>, rota::Int4Smem<64>::ALLOC, grid, s, p);
   return st;
 }
 
 rota_status rota_attn_fwd_int4(const rota_attn_desc* d, const rota_attn_buffers* buf, const uint8_t* head_flags,
                                float* out, void* stream) {
   return launch_int4(d, buf, head_flags, out, stream, false, 0, 0, 0, 0, nullptr, nullptr);
+}
+
+rota_status rota_attn_int4_widen(const rota_attn_desc* d, const rota_attn_buffers* buf, const uint8_t* head_flags,
+                                 void* stream) {
+  return launch_int4(d, buf, head_flags, nullptr, stream, false, 0, 0, 0, 0, nullptr, nullptr, 1);
+}
+
+rota_status rota_attn_int4_attend(const rota_attn_desc* d, const rota_attn_buffers* buf, const uint8_t* head_flags,
+                                  float* out, void* stream) {
+  return launch_int4(d, buf, head_flags, out, stream, false, 0, 0, 0, 0, nullptr, nullptr, 2);
 }
 
 rota_status rota_attn_debug_dump_int4(const rota_attn_desc* d, const rota_attn_buffers* buf, int32_t b, int32_t h,

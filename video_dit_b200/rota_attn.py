@@ -54,6 +54,8 @@ _SIGS = {
     "rota_attn_build_rope_tables": ([_D, _P, _P], ctypes.c_int),
     "rota_attn_prepare_qk": ([_D, _P, _P, _P, _P, _BUF, _P], ctypes.c_int),
     "rota_attn_fwd_int4": ([_D, _BUF, _P, _P, _P], ctypes.c_int),
+    "rota_attn_int4_widen": ([_D, _BUF, _P, _P], ctypes.c_int),
+    "rota_attn_int4_attend": ([_D, _BUF, _P, _P, _P], ctypes.c_int),
     "rota_attn_fwd_fp16_fallback": ([_D, _BUF, _P, _P, _P, _P], ctypes.c_int),
     "rota_attn_get_error": ([_P], ctypes.c_int),
     "rota_attn_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -142,6 +144,15 @@ def rota_attn_prepare_qk(desc, q, k, v, head_flags, buffers: rota_attn_buffers, 
 def rota_attn_fwd_int4(desc, buffers: rota_attn_buffers, head_flags, out, stream=None) -> int:
     return _lib.rota_attn_fwd_int4(ctypes.byref(desc), ctypes.byref(buffers), _flags(head_flags), _ptr(out),
                                    _stream(stream))
+
+
+def rota_attn_int4_widen(desc, buffers: rota_attn_buffers, head_flags, stream=None) -> int:
+    return _lib.rota_attn_int4_widen(ctypes.byref(desc), ctypes.byref(buffers), _flags(head_flags), _stream(stream))
+
+
+def rota_attn_int4_attend(desc, buffers: rota_attn_buffers, head_flags, out, stream=None) -> int:
+    return _lib.rota_attn_int4_attend(ctypes.byref(desc), ctypes.byref(buffers), _flags(head_flags), _ptr(out),
+                                      _stream(stream))
 
 
 def rota_attn_fwd_fp16_fallback(desc, buffers: rota_attn_buffers, v, head_flags, out, stream=None) -> int:
@@ -367,7 +378,3 @@ class RotaAttention:
             k_rope=None if self.k_rope is None else self.k_rope[: B * H * N * D * 2].view(torch.int16).view(B, H, N, D),
         )
 
-
-def kappa(head_dim: int, sm_scale: float = 0.0) -> float:
-    s = np.float32(sm_scale) if sm_scale > 0 else np.float32(1.0 / math.sqrt(head_dim))
-    return float(np.float32(np.float64(s) * 1.4426950408889634))
