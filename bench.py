@@ -156,7 +156,8 @@ def oracle_sample(w, q, k, v, rows: int = 128):
     prep = oracle.prepare(qs, ks, vs, w.grid, w.rope_dim, w.had_block, w.theta, flags, phase=w.rope_phase)
     t1 = time.perf_counter()
     r0 = max(0, w.N // 2 - rows // 2)
-    oracle.attn_int4(prep, w.N, float(np.float32(1 / np.sqrt(w.d))), 0, 0, r0, rows)
+    oracle.attn_int4(prep, w.N, float(np.float32(1 / np.sqrt(w.d))), 0, 0, r0, rows, group=w.max_group,
+                     rowsum=w.row_sum)
     t2 = time.perf_counter()
     t_prep_full = (t1 - t0) * w.B * w.H
     t_attn_full = (t2 - t1) * (w.B * w.H * w.N / rows)
@@ -180,7 +181,7 @@ def accuracy_sample(w, q, k, v, out, h, rows):
     r0 = max(0, w.N // 2 - rows // 2)
     prep = oracle.prepare(qs, ks, vs, w.grid, w.rope_dim, w.had_block, w.theta, np.zeros(1, np.uint8),
                           phase=w.rope_phase)
-    o4 = oracle.attn_int4(prep, w.N, sm, 0, 0, r0, rows)
+    o4 = oracle.attn_int4(prep, w.N, sm, 0, 0, r0, rows, group=w.max_group, rowsum=w.row_sum)
     unq = oracle.attn_ref(qs, ks, vs, w.grid, w.rope_dim, sm, 0, 0, r0, rows, theta=w.theta, phase=w.rope_phase)
     got = out[0, h, r0:r0 + rows].double().cpu().numpy()
     err = np.abs(got - o4)
@@ -261,7 +262,8 @@ def main():
     flags = w.flags()
     qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
     qd, kd, vd = (x.to(dev) for x in (qh, kh, vh))
-    desc = ra.make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta, rope_phase=w.rope_phase)
+    desc = ra.make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta, rope_phase=w.rope_phase,
+                        max_group=w.max_group, row_sum=w.row_sum)
     att = ra.RotaAttention(desc, device=dev, need_fp16=bool(flags.any()))
     out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device=dev)
     out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()

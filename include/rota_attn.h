@@ -71,6 +71,17 @@ typedef enum {
  *   applied to Q and K alike and free at run time (it lives in the tables).
  *   0 = plain RoPE.  It composes with had_block (rotation after RoPE).
  * head_dim: 64 or 128.
+ * quant_block: tokens per Q / K / V quantisation block; 0 or 64 (the only
+ *   size implemented; anything else positive is ROTA_ERR_UNSUPPORTED).
+ * max_group: keys per group of the running max the P codes are taken
+ *   against (the codes of a group use the max over every key up to its
+ *   end): 0 or 64 (= the quantisation block) or 128 (two blocks share one
+ *   max); other positive values are ROTA_ERR_UNSUPPORTED.
+ * row_sum: the softmax row sum l.  0: the sum of the P codes u (the values
+ *   that multiply V, so the 1/15 scale cancels); 1: the sum of the
+ *   unquantised 15 * 2^d the codes are rounded from.
+ * A zeroed field selects the default (quant_block 64, max_group 64,
+ * row_sum 0).
  */
 typedef struct {
   int32_t B, H, N, head_dim;
@@ -80,6 +91,9 @@ typedef struct {
   float rope_theta;
   float sm_scale;
   float rope_phase[3];
+  int32_t quant_block;
+  int32_t max_group;
+  int32_t row_sum;
 } rota_attn_desc;
 
 /*

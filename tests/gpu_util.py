@@ -16,7 +16,8 @@ def lib():
 
 
 def desc_of(w: synth.Workload):
-    return lib().make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta, rope_phase=w.rope_phase)
+    return lib().make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta, rope_phase=w.rope_phase,
+                        max_group=w.max_group, row_sum=w.row_sum)
 
 
 def to_dev(a: np.ndarray):

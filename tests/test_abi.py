@@ -38,7 +38,8 @@ def test_every_declared_symbol_is_exported(ra):
 
 
 def _desc(ra, w):
-    return ra.make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta, rope_phase=w.rope_phase)
+    return ra.make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta, rope_phase=w.rope_phase,
+                        max_group=w.max_group, row_sum=w.row_sum)
 
 
 def test_validate_accepts_workloads(ra):
@@ -49,11 +50,21 @@ def test_validate_accepts_workloads(ra):
 @pytest.mark.parametrize("field,value,status", [
     ("N", 1000, 1), ("head_dim", 96, 1), ("B", 0, 1), ("grid_w", 0, 1),
     ("rope_theta", -1.0, 1), ("sm_scale", float("nan"), 1), ("H", 300, 2),
+    ("quant_block", 32, 2), ("quant_block", -64, 1), ("max_group", 256, 2), ("max_group", 96, 2),
+    ("max_group", -1, 1), ("row_sum", 2, 1), ("row_sum", -1, 1),
 ])
 def test_validate_rejects(ra, field, value, status):
     d = _desc(ra, synth.WORKLOADS["wan480"])
     setattr(d, field, value)
     assert ra.rota_attn_validate(d) == status
+
+
+@pytest.mark.parametrize("field,value", [("quant_block", 0), ("quant_block", 64), ("max_group", 0), ("max_group", 64),
+                                         ("max_group", 128), ("row_sum", 0), ("row_sum", 1)])
+def test_validate_accepts_numerics_options(ra, field, value):
+    d = _desc(ra, synth.WORKLOADS["wan480"])
+    setattr(d, field, value)
+    assert ra.rota_attn_validate(d) == ra.ROTA_OK
 
 
 def test_validate_rejects_bad_partitions(ra):

@@ -63,7 +63,7 @@ def test_edge_case_parity(case):
         assert np.array_equal(codes[key], ref[key]), key
     for key in ("q_scale", "k_scale", "v_scale"):
         assert np.array_equal(codes[key].view(np.uint32), ref[key].view(np.uint32)), key
-    o_ref, s_ref, p_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, 0, w.N, dump=True)
+    o_ref, s_ref, p_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, 0, w.N, dump=True, group=w.max_group, rowsum=w.row_sum)
     if case == "huge":
         kappa = np.float64(np.float32(np.float64(np.float32(sm_scale(w))) * 1.4426950408889634))
         cmax = np.float64(ref["q_scale"].max()) * np.float64(ref["k_scale"].max()) * kappa
@@ -72,7 +72,7 @@ def test_edge_case_parity(case):
     assert np.array_equal(p, p_ref)
     heads = range(w.H) if w.H <= 8 else (0, 1, w.H // 2, w.H - 1)
     for hh in heads:
-        o = o_ref if hh == h else oracle.attn_int4(ref, w.N, sm_scale(w), 0, hh, 0, w.N)
+        o = o_ref if hh == h else oracle.attn_int4(ref, w.N, sm_scale(w), 0, hh, 0, w.N, group=w.max_group, rowsum=w.row_sum)
         assert np.isfinite(out[0, hh]).all(), hh
         e, rel, cos = row_stats(out[0, hh], o)
         assert e <= TOL, (hh, e, rel, cos)

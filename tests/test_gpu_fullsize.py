@@ -51,7 +51,7 @@ def _int4_full_size(name, code_heads, h, tiles):
         scratch = torch.empty_like(out)
         ra._check(ra.rota_attn_debug_dump_int4(att.desc, att.buffers, 0, h, r0, nr, s, p, scratch), "dump")
         assert ra.rota_attn_get_error() == ra.ROTA_OK
-        o_ref, s_ref, p_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, 0, r0, nr, dump=True)
+        o_ref, s_ref, p_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, 0, r0, nr, dump=True, group=w.max_group, rowsum=w.row_sum)
         assert np.array_equal(s.cpu().numpy(), s_ref)
         assert np.array_equal(p.cpu().numpy(), p_ref)
         got = out[0, h, r0:r0 + nr].cpu().numpy()
@@ -92,6 +92,6 @@ def test_wan720_mixed_precision_sampled_rows():
     h = 11
     ref = oracle.prepare(_head(q, h), _head(k, h), _head(v, h), w.grid, w.rope_dim, w.had_block, w.theta)
     for r0, nr in ((w.N // 3, 32), (w.N - 16, 16)):
-        o4 = oracle.attn_int4(ref, w.N, sm_scale(w), 0, 0, r0, nr)
+        o4 = oracle.attn_int4(ref, w.N, sm_scale(w), 0, 0, r0, nr, group=w.max_group, rowsum=w.row_sum)
         e, rel, cos = row_stats(out[0, h, r0:r0 + nr].cpu().numpy(), o4)
         assert e <= TOL, (r0, e, rel, cos)

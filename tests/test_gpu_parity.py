@@ -35,6 +35,13 @@ CASES = {
     # q = 43) and the 56-channel ones (Paley II, q = 13, doubled)
     "hadamard_44": synth.scaled(synth.WORKLOADS["wan480"], "h44", H=2, grid=(3, 10, 13), had=(44, 2, 2)),
     "hadamard_56": synth.scaled(synth.WORKLOADS["hunyuan"], "h56", H=2, grid=(3, 9, 20), had=(16, 56, 56)),
+    # numerics options: the running max over 128-key groups (two blocks share one max; an odd
+    # block count leaves a one-block last group), and the unquantised row sum l = sum 15 * 2^d
+    "max_group_128": synth.scaled(synth.WORKLOADS["wan480"], "g128", H=2, grid=(3, 10, 13), max_group=128),
+    "max_group_128_even": synth.scaled(synth.WORKLOADS["hunyuan"], "g128e", H=2, grid=(2, 8, 16),
+                                       max_group=128),
+    "row_sum_r1": synth.scaled(synth.WORKLOADS["wan480"], "r1", H=2, grid=(3, 10, 13), row_sum=1),
+    "g128_r1_tiny": synth.scaled(synth.WORKLOADS["tiny"], "g128r1", max_group=128, row_sum=1),
 }
 
 # Many key blocks per CTA (74), so every pipeline stage and barrier phase wraps many times.
@@ -65,7 +72,7 @@ def test_int4_scores_and_pcodes_bit_exact(name):
     r0, nr = (0, w.N) if w.N <= 400 else (w.N - 150, 150)
     _, out, (s, p, _) = run(w, q, k, v, dump=(0, h, r0, nr))
     ref = _oracle(w, q, k, v)
-    o_ref, s_ref, p_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, r0, nr, dump=True)
+    o_ref, s_ref, p_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, r0, nr, dump=True, group=w.max_group, rowsum=w.row_sum)
     assert np.array_equal(s, s_ref)
     assert np.array_equal(p, p_ref)
     e, rel, cos = row_stats(out[0, h, r0:r0 + nr], o_ref)
@@ -80,7 +87,7 @@ def test_int4_output_all_heads(name):
     _, out, _ = run(w, q, k, v)
     ref = _oracle(w, q, k, v)
     for h in range(w.H):
-        o_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, 0, w.N)
+        o_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, 0, w.N, group=w.max_group, rowsum=w.row_sum)
         e, rel, cos = row_stats(out[0, h], o_ref)
         assert e <= TOL, (h, e, rel, cos)
 
@@ -99,7 +106,7 @@ def test_fp16_fallback_heads(name):
     e, rel, cos = row_stats(out[0, 0], o16)
     assert e <= TOL, (e, rel, cos)
     for h in range(1, w.H):          # the INT4 heads of the same call are unaffected
-        o_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, 0, w.N)
+        o_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, 0, w.N, group=w.max_group, rowsum=w.row_sum)
         assert row_stats(out[0, h], o_ref)[0] <= TOL
 
 
@@ -143,13 +150,13 @@ def test_int4_long_sequence_sampled_rows():
     h, r0, nr = 1, w.N - 200, 200          # the last two CTAs of the head, ragged tail included
     _, out, (s, p, _) = run(w, q, k, v, dump=(0, h, r0, nr))
     ref = _oracle(w, q, k, v)
-    o_ref, s_ref, p_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, r0, nr, dump=True)
+    o_ref, s_ref, p_ref = oracle.attn_int4(ref, w.N, sm_scale(w), 0, h, r0, nr, dump=True, group=w.max_group, rowsum=w.row_sum)
     assert np.array_equal(s, s_ref)
     assert np.array_equal(p, p_ref)
     e, rel, cos = row_stats(out[0, h, r0:r0 + nr], o_ref)
     report(f"parity/long h{h}", accuracy(w, q, k, v, out[0, h, r0:r0 + nr], o_ref, 0, h, r0, nr))
     assert e <= TOL, (e, rel, cos)
-    o0 = oracle.attn_int4(ref, w.N, sm_scale(w), 0, 0, 0, 64)          # first rows of the other head
+    o0 = oracle.attn_int4(ref, w.N, sm_scale(w), 0, 0, 0, 64, group=w.max_group, rowsum=w.row_sum)          # first rows of the other head
     assert row_stats(out[0, 0, :64], o0)[0] <= TOL
 
 

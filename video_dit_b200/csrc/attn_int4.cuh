@@ -72,6 +72,7 @@ struct Int4Params {
   int32_t* s_dump;
   uint8_t* p_dump;
   int dbg_r0, dbg_nr;
+  int row_sum;          // 0: l sums the codes; 1: l sums the unquantised 15 * 2^d
 };
 
 constexpr int kInt4Threads = 512;
@@ -87,8 +88,11 @@ constexpr int kLaunchRegs = (128 * kIssueRegs + 256 * kSoftmaxRegs + 128 * kCorr
 static_assert(kLaunchRegs * 512 == 128 * kIssueRegs + 256 * kSoftmaxRegs + 128 * kCorrRegs, "register split");
 static_assert(kLaunchRegs == 128, "launch allocation");
 
-template <int D>
+template <int D, int G = 64>
 struct Int4Smem {
+  // 128-key groups keep a block's scores in shared memory until the next
+  // block's are in (the spill area), paid for with two fewer operand stages
+  static constexpr int OPS = G == 128 ? kOps - 2 : kOps;
   static constexpr uint32_t LAYOUT_QK = D == 128 ? 2u : 4u;  // 128B / 64B swizzle of the Q and K rows
   static constexpr uint32_t SBO_QK = 8 * D;
   static constexpr int Q_BYTES = kBM * D;         // one tile, e4m3
@@ -100,14 +104,16 @@ struct Int4Smem {
   static constexpr int OFF_Q = 0;                                 // [tile]
   static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;               // [tile][slot]
   static constexpr int OFF_OP = OFF_P + 4 * P_BYTES;              // [stage]
-  static constexpr int OFF_ALPHA = OFF_OP + kOps * OP_BYTES;      // float [tile][slot][128]
+  static constexpr int OFF_ALPHA = OFF_OP + OPS * OP_BYTES;       // float [tile][slot][128]
   static constexpr int OFF_FLAG = OFF_ALPHA + 4 * kBM * 4;        // int [tile][slot][4 warps]
   static constexpr int OFF_L = OFF_FLAG + 16 * 4;                 // float [tile][128]
   static constexpr int OFF_TAU = OFF_L + 2 * kBM * 4;
-  static constexpr int OFF_BAR = OFF_TAU + 64;
-  // barriers: op_full[kOps] op_empty[kOps] q_full s_full[2] s_empty[2]
+  static constexpr int OFF_SPILL = OFF_TAU + 64;                  // float4 [tile][16][128] (G = 128)
+  static constexpr int SPILL_BYTES = G == 128 ? 2 * kBM * kBN * 4 : 0;
+  static constexpr int OFF_BAR = OFF_SPILL + SPILL_BYTES;
+  // barriers: op_full[OPS] op_empty[OPS] q_full s_full[2] s_empty[2]
   //           p_full[2][2] p_empty[2][2] acc_full acc_empty l_full mma_done[2]
-  static constexpr int NBAR = 2 * kOps + 1 + 2 + 2 + 4 + 4 + 1 + 1 + 1 + 2;
+  static constexpr int NBAR = 2 * OPS + 1 + 2 + 2 + 4 + 4 + 1 + 1 + 1 + 2;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int BYTES = OFF_ABORT + 4;
@@ -117,6 +123,8 @@ struct Int4Smem {
   static_assert(T_ACC + kBM <= T_O && T_O + 2 * kBM <= TMEM_COLS, "TMEM budget");
   static_assert(D <= 128, "one TMEM lane per channel");
   static_assert(IMG_BYTES % 16 == 0 && K_BYTES % 16 == 0 && VT_BYTES % 16 == 0, "bulk copy sizes");
+  static_assert(G == 64 || G == 128, "max group");
+  static_assert(OFF_SPILL % 16 == 0, "spill alignment");
   static_assert(OFF_P % 1024 == 0 && OFF_OP % 1024 == 0 && OP_BYTES % 1024 == 0 && K_BYTES % 1024 == 0 &&
                     P_BYTES % 1024 == 0,
                 "swizzle atom alignment");
@@ -156,13 +164,10 @@ __device__ __forceinline__ void setmaxnreg_corr() {
 }
 static_assert(kIssueRegs == 32 && kSoftmaxRegs == 136 && kCorrRegs == 208, "setmaxnreg immediates");
 
-// One 64-key block of one softmax thread: the running max, the P codes as
-// bytes (4 per word, key 4w + i in byte i of word w) and their sum.  S holds
-// the block's scores S_int * 2^-18; keys >= nvalid (MASK) take code 0 and do
-// not enter the max.  Returns the code sum; m is updated.
+// The max of one 64-key block's scores S = S_int * 2^-18 over the valid keys;
+// keys >= nvalid (MASK) are set to -inf in sr, so they never enter a max.
 template <bool MASK>
-__device__ __forceinline__ uint32_t block_codes(uint32_t (&sr)[kBN], int nvalid, float c18, float& m,
-                                                uint32_t (&pw)[kBN / 4], const float* tau) {
+__device__ __forceinline__ float block_max(uint32_t (&sr)[kBN], int nvalid) {
   if (MASK) {
 #pragma unroll
     for (int k = 0; k < kBN; ++k)
@@ -176,9 +181,19 @@ __device__ __forceinline__ uint32_t block_codes(uint32_t (&sr)[kBN], int nvalid,
     x2 = max3(x2, __uint_as_float(sr[k + 4]), __uint_as_float(sr[k + 5]));
     x3 = max3(x3, __uint_as_float(sr[k + 6]), __uint_as_float(sr[k + 7]));
   }
-  const float smax = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
-  m = fmaxf(m, __fmul_rn(smax, c18));
+  return fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+}
+
+// The P codes of one 64-key block of one softmax thread against the group
+// max m: bytes, 4 per word (key 4w + i in byte i of word w), keys >= nvalid
+// (MASK) code 0.  Returns the sum of the codes; with R1, lsum also receives
+// the row-sum term 15 * sum_k 2^d_k (the unquantised values the codes are
+// rounded from, from the same exponentials).
+template <bool MASK, bool R1>
+__device__ __forceinline__ uint32_t block_codes(const uint32_t (&sr)[kBN], int nvalid, float c18, float m,
+                                                uint32_t (&pw)[kBN / 4], const float* tau, float& lsum) {
   uint32_t sum_lo = 0, sum_hi = 0;
+  float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
   for (int k = 0; k < kBN; k += 4) {
     float d0, d1, d2, d3;
@@ -200,7 +215,12 @@ __device__ __forceinline__ uint32_t block_codes(uint32_t (&sr)[kBN], int nvalid,
     sum_hi += __float_as_uint(h0) + __float_as_uint(h1) + __float_as_uint(h2) + __float_as_uint(h3);
     pw[k / 4] = prmt(prmt(__float_as_uint(l0), __float_as_uint(l1), 0x0040u),
                      prmt(__float_as_uint(l2), __float_as_uint(l3), 0x0040u), 0x5410u);
+    if (R1) {
+      add2(ls0, ls1, ls0, ls1, e0, e1);
+      add2(ls0, ls1, ls0, ls1, e2, e3);
+    }
   }
+  if (R1) lsum = __fmul_rn(15.f, __fadd_rn(ls0, ls1));
   // 64 kMag bit patterns sum to 0xC0000000 (mod 2^32)
   uint32_t usum = sum_lo - 0xC0000000u;
   // Exact decisions (rare): some key of the warp's rows lies in the band
@@ -227,9 +247,23 @@ __device__ __forceinline__ uint32_t block_codes(uint32_t (&sr)[kBN], int nvalid,
   return usum;
 }
 
-template <int D>
+// The codes of one block with the row-sum reading chosen at run time; returns
+// the block's contribution to l (the code sum, or 15 sum 2^d).
+template <bool MASK>
+__device__ __forceinline__ float block_codes_l(const uint32_t (&sr)[kBN], int nvalid, float c18, float m,
+                                               uint32_t (&pw)[kBN / 4], const float* tau, bool r1) {
+  float lsum = 0.f;
+  if (r1) {
+    block_codes<MASK, true>(sr, nvalid, c18, m, pw, tau, lsum);
+    return lsum;
+  }
+  return static_cast<float>(block_codes<MASK, false>(sr, nvalid, c18, m, pw, tau, lsum));
+}
+
+template <int D, int G>
 __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid_constant__ Int4Params p) {
-  using L = Int4Smem<D>;
+  using L = Int4Smem<D, G>;
+  constexpr int kOps = L::OPS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
@@ -421,53 +455,38 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     }
     const float sq = row < npad ? __ldg(p.q_scale + head * p.nblk + row / kBN) : 0.f;
     const float* ksc = p.k_scale + head * p.nblk;
-    const bool dump_rows = p.s_dump != nullptr;
+    const bool dump_rows = p.s_dump != nullptr && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr;
+    const bool r1 = p.row_sum != 0;
 
-    float m = -INFINITY, l = 0.f;
-    bool aborted = false;
-    float sk_next = __ldg(ksc);
-    for (int j = 0; j < nkb; ++j) {
-      const float sk = sk_next;
-      if (j + 1 < nkb) sk_next = __ldg(ksc + j + 1);
-      const int sl = j & 1;
-      if (!warp_wait(&s_full[t], j & 1, lim)) { aborted = true; break; }
+    // S of block j -> registers; the buffer is released at once, so the MMA
+    // computes the tile's next scores while these are coded
+    auto load_s = [&](int j, uint32_t (&sr)[kBN]) -> bool {
+      if (!warp_wait(&s_full[t], j & 1, lim)) return false;
       tc_fence_after();
-      const int nvalid = min(kBN, p.N - j * kBN);
-      const float c18 = __fmul_rn(__fmul_rn(__fmul_rn(sq, sk), p.kappa), 262144.f);  // S = S_int 2^-18
-      uint32_t sr[kBN];
-      {
-        uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-        uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        tmem_ld32(tS, s0);
-        tmem_ld32(tS + 32, s1);
-        tmem_wait_dep2(s0, s1);
-      }
-      // S is in registers: the MMA may compute S(j+1) into this buffer now
+      uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+      uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+      tmem_ld32(tS, s0);
+      tmem_ld32(tS + 32, s1);
+      tmem_wait_dep2(s0, s1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[t]);
-      if (dump_rows && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr) {
+      if (__any_sync(0xffffffffu, dump_rows)) {
+        const int nvalid = min(kBN, p.N - j * kBN);
 #pragma unroll
         for (int k = 0; k < kBN; ++k)
-          if (k < nvalid)
+          if (dump_rows && k < nvalid)
             p.s_dump[(size_t)(row - p.dbg_r0) * p.N + (size_t)j * kBN + k] =
                 static_cast<int32_t>(__uint_as_float(sr[k]) * 262144.f);
       }
-      const float m_old = m;
-      uint32_t pw[kBN / 4];
-      const uint32_t usum = nvalid == kBN ? block_codes<false>(sr, nvalid, c18, m, pw, sTau)
-                                          : block_codes<true>(sr, nvalid, c18, m, pw, sTau);
-      // alpha = 2^(m_old - m) for the rows whose max moved (exact 1 elsewhere)
-      float alpha = 0.f;
-      if (j > 0) {
-        alpha = 1.f;
-        if (__any_sync(0xffffffffu, m != m_old))
-          if (m != m_old) alpha = exp2f(m_old - m);
-      }
-      l = __fmaf_rn(l, alpha, static_cast<float>(usum));
-
+      return true;
+    };
+    // the codes of block j -> its P slot (the B operand of P V), with alpha
+    // (the factor on O before the block is added) and the warp's flag
+    auto emit = [&](int j, const uint32_t (&pw)[kBN / 4], float alpha) -> bool {
+      const int sl = j & 1;
       // the slot's previous codes (block j - 2) are consumed
-      if (j >= 2 && !warp_wait(&p_empty[2 * t + sl], ((j >> 1) & 1) ^ 1, lim)) { aborted = true; break; }
+      if (j >= 2 && !warp_wait(&p_empty[2 * t + sl], ((j >> 1) & 1) ^ 1, lim)) return false;
       uint8_t* sP = smem + L::OFF_P + (2 * t + sl) * L::P_BYTES;
 #pragma unroll
       for (int i = 0; i < kBN / 16; ++i)
@@ -476,17 +495,104 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       sAlpha[(2 * t + sl) * kBM + r] = alpha;
       const bool moved = __any_sync(0xffffffffu, alpha != 1.f);
       if (lane == 0) sFlag[(2 * t + sl) * 4 + (warp & 3)] = moved ? 1 : 0;
-      if (dump_rows && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr) {
+      if (__any_sync(0xffffffffu, dump_rows)) {
+        const int nvalid = min(kBN, p.N - j * kBN);
 #pragma unroll
         for (int k = 0; k < kBN; ++k)
-          if (k < nvalid)
+          if (dump_rows && k < nvalid)
             p.p_dump[(size_t)(row - p.dbg_r0) * p.N + (size_t)j * kBN + k] =
                 static_cast<uint8_t>((pw[k >> 2] >> (8 * (k & 3))) & 0xFFu);
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[2 * t + sl]);
-      if (warp_flag(sAbort)) { aborted = true; break; }
+      return true;
+    };
+    // alpha = 2^(m_old - m) for the rows whose max moved (exact 1 elsewhere; 0
+    // before the first block, where O is not read)
+    auto alpha_of = [&](bool first, float m_old, float m_new) -> float {
+      if (first) return 0.f;
+      float alpha = 1.f;
+      if (__any_sync(0xffffffffu, m_new != m_old))
+        if (m_new != m_old) alpha = exp2f(m_old - m_new);
+      return alpha;
+    };
+    auto c18_of = [&](float sk) {   // S = S_int 2^-18, so c * 2^18 (exact) multiplies S
+      return __fmul_rn(__fmul_rn(__fmul_rn(sq, sk), p.kappa), 262144.f);
+    };
+    // the key scales are read one block (pair) ahead
+    float sk_next = __ldg(ksc), sk_next2 = nkb > 1 ? __ldg(ksc + 1) : 0.f;
+
+    float m = -INFINITY, l = 0.f;
+    bool aborted = false;
+    if constexpr (G == 64) {
+      for (int j = 0; j < nkb; ++j) {
+        const float c18 = c18_of(sk_next);
+        if (j + 1 < nkb) sk_next = __ldg(ksc + j + 1);
+        uint32_t sr[kBN];
+        if (!load_s(j, sr)) { aborted = true; break; }
+        const int nvalid = min(kBN, p.N - j * kBN);
+        const float smax = nvalid == kBN ? block_max<false>(sr, nvalid) : block_max<true>(sr, nvalid);
+        const float m_old = m;
+        m = fmaxf(m, __fmul_rn(smax, c18));
+        uint32_t pw[kBN / 4];
+        const float lsum = nvalid == kBN ? block_codes_l<false>(sr, nvalid, c18, m, pw, sTau, r1)
+                                         : block_codes_l<true>(sr, nvalid, c18, m, pw, sTau, r1);
+        const float alpha = alpha_of(j == 0, m_old, m);
+        l = __fmaf_rn(l, alpha, lsum);
+        if (!emit(j, pw, alpha)) { aborted = true; break; }
+        if (warp_flag(sAbort)) { aborted = true; break; }
+      }
+    } else {
+      // 128-key groups: blocks j0 = 2g and j1 = 2g + 1 share the max over both,
+      // so block j0's scores wait in shared memory while j1's come in; j1 is
+      // coded first (from registers), then j0 (reloaded)
+      float4* spill = reinterpret_cast<float4*>(smem + L::OFF_SPILL) + t * (kBN / 4) * kBM;
+      for (int j0 = 0; j0 < nkb; j0 += 2) {
+        const int j1 = j0 + 1;
+        const bool has1 = j1 < nkb;
+        const float c0 = c18_of(sk_next);
+        const float c1 = has1 ? c18_of(sk_next2) : 0.f;
+        if (j0 + 2 < nkb) sk_next = __ldg(ksc + j0 + 2);
+        if (j0 + 3 < nkb) sk_next2 = __ldg(ksc + j0 + 3);
+        const int nv0 = min(kBN, p.N - j0 * kBN), nv1 = has1 ? min(kBN, p.N - j1 * kBN) : 0;
+        uint32_t sr[kBN];
+        if (!load_s(j0, sr)) { aborted = true; break; }
+        const float smax0 = nv0 == kBN ? block_max<false>(sr, nv0) : block_max<true>(sr, nv0);
+#pragma unroll
+        for (int i = 0; i < kBN / 4; ++i)
+          spill[i * kBM + r] = make_float4(__uint_as_float(sr[4 * i]), __uint_as_float(sr[4 * i + 1]),
+                                           __uint_as_float(sr[4 * i + 2]), __uint_as_float(sr[4 * i + 3]));
+        float x1 = -INFINITY;
+        if (has1) {
+          if (!load_s(j1, sr)) { aborted = true; break; }
+          const float smax1 = nv1 == kBN ? block_max<false>(sr, nv1) : block_max<true>(sr, nv1);
+          x1 = __fmul_rn(smax1, c1);
+        }
+        const float m_old = m;
+        m = fmaxf(fmaxf(m, __fmul_rn(smax0, c0)), x1);
+        const float alpha = alpha_of(j0 == 0, m_old, m);
+        uint32_t pw[kBN / 4];
+        float lsum1 = 0.f;
+        if (has1) {
+          lsum1 = nv1 == kBN ? block_codes_l<false>(sr, nv1, c1, m, pw, sTau, r1)
+                             : block_codes_l<true>(sr, nv1, c1, m, pw, sTau, r1);
+          if (!emit(j1, pw, 1.f)) { aborted = true; break; }
+        }
+#pragma unroll
+        for (int i = 0; i < kBN / 4; ++i) {
+          const float4 x = spill[i * kBM + r];
+          sr[4 * i] = __float_as_uint(x.x);
+          sr[4 * i + 1] = __float_as_uint(x.y);
+          sr[4 * i + 2] = __float_as_uint(x.z);
+          sr[4 * i + 3] = __float_as_uint(x.w);
+        }
+        const float lsum0 = nv0 == kBN ? block_codes_l<false>(sr, nv0, c0, m, pw, sTau, r1)
+                                       : block_codes_l<true>(sr, nv0, c0, m, pw, sTau, r1);
+        l = __fadd_rn(__fmaf_rn(l, alpha, lsum0), lsum1);
+        if (!emit(j0, pw, alpha)) { aborted = true; break; }
+        if (warp_flag(sAbort)) { aborted = true; break; }
+      }
     }
     if (aborted) *sAbort = 1;
     sL[t * kBM + r] = l;
@@ -619,7 +725,7 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
 // rows x 64 keys of e4m3 subnormals (64B swizzle; rows >= D are zero).
 template <int D>
 __global__ void __launch_bounds__(256) widen_kv_kernel(const __grid_constant__ Int4Params p, uint8_t* work) {
-  using L = Int4Smem<D>;
+  using L = Int4Smem<D, 64>;   // the images do not depend on the max group
   const int j = blockIdx.x, h = p.heads[blockIdx.y], b = blockIdx.z;
   const size_t head = (size_t)b * p.H + h;
   const int npad = p.nblk * kBN;

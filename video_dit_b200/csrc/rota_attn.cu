@@ -267,7 +267,10 @@ rota_status rota_attn_validate(const rota_attn_desc* d) {
   if (!(d->sm_scale >= 0.f) || !std::isfinite(d->sm_scale)) return ROTA_ERR_INVALID_ARG;
   for (int a = 0; a < 3; ++a)
     if (!std::isfinite(d->rope_phase[a])) return ROTA_ERR_INVALID_ARG;
+  if (d->quant_block < 0 || d->max_group < 0 || d->row_sum < 0 || d->row_sum > 1) return ROTA_ERR_INVALID_ARG;
   if (d->head_dim != 64 && d->head_dim != 128) return ROTA_ERR_UNSUPPORTED;
+  if (d->quant_block != 0 && d->quant_block != 64) return ROTA_ERR_UNSUPPORTED;
+  if (d->max_group != 0 && d->max_group != 64 && d->max_group != 128) return ROTA_ERR_UNSUPPORTED;
   if (d->H > 256) return ROTA_ERR_UNSUPPORTED;
   if (static_cast<long long>(d->B) * d->H * npad_of(d->N) * d->head_dim > (1ll << 40)) return ROTA_ERR_UNSUPPORTED;
   if (d->B > 65535) return ROTA_ERR_UNSUPPORTED;
@@ -291,7 +294,7 @@ rota_status rota_attn_buffer_sizes(const rota_attn_desc* d, size_t* bytes) {
   bytes[ROTA_BUF_ROPE_TABLE] = 4 * (static_cast<size_t>(d->grid_t) * (d->rope_dim[0] / 2) +
                                     static_cast<size_t>(d->grid_h) * (d->rope_dim[1] / 2) +
                                     static_cast<size_t>(d->grid_w) * (d->rope_dim[2] / 2));
-  bytes[ROTA_BUF_INT4_WORK] = heads * nblk * (D == 128 ? rota::Int4Smem<128>::IMG_BYTES : rota::Int4Smem<64>::IMG_BYTES);
+  bytes[ROTA_BUF_INT4_WORK] = heads * nblk * (D == 128 ? rota::Int4Smem<128, 64>::IMG_BYTES : rota::Int4Smem<64, 64>::IMG_BYTES);
   return ROTA_OK;
 }
 
@@ -402,6 +405,7 @@ static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers*
   p.N = d->N;
   p.nblk = npad_of(d->N) / 64;
   p.kappa = kappa_of(d);
+  p.row_sum = d->row_sum;
   std::memcpy(p.tau, tau_table().tau, sizeof(p.tau));
   {
     std::lock_guard<std::mutex> g(g_inject.mu);
@@ -429,7 +433,7 @@ static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers*
     p.k_scale += hs * nblk;
     p.v_codes += hs * nblk * D * 32;
     p.v_scale += hs * nblk * D;
-    p.work += hs * nblk * (D == 128 ? rota::Int4Smem<128>::IMG_BYTES : rota::Int4Smem<64>::IMG_BYTES);
+    p.work += hs * nblk * (D == 128 ? rota::Int4Smem<128, 64>::IMG_BYTES : rota::Int4Smem<64, 64>::IMG_BYTES);
     p.out += hs * d->N * D;
   } else {
     p.nheads = select_heads(d, head_flags, 0, p.heads);
@@ -449,10 +453,13 @@ static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers*
   // 2. attention
   const dim3 grid((d->N + rota::kRowsPerCta - 1) / rota::kRowsPerCta, p.nheads, batches);
   // the debug dump runs the same kernel with its dump pointers set
+  const bool g128 = d->max_group == 128;
   if (d->head_dim == 128)
-    st = launch_int4_kernel(rota::attn_int4_kernel<128>, rota::Int4Smem<128>::ALLOC, grid, s, p);
+    st = g128 ? launch_int4_kernel(rota::attn_int4_kernel<128, 128>, rota::Int4Smem<128, 128>::ALLOC, grid, s, p)
+              : launch_int4_kernel(rota::attn_int4_kernel<128, 64>, rota::Int4Smem<128, 64>::ALLOC, grid, s, p);
   else
-    st = launch_int4_kernel(rota::attn_int4_kernel<64>, rota::Int4Smem<64>::ALLOC, grid, s, p);
+    st = g128 ? launch_int4_kernel(rota::attn_int4_kernel<64, 128>, rota::Int4Smem<64, 128>::ALLOC, grid, s, p)
+              : launch_int4_kernel(rota::attn_int4_kernel<64, 64>, rota::Int4Smem<64, 64>::ALLOC, grid, s, p);
   return st;
 }
 

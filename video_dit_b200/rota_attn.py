@@ -33,7 +33,8 @@ class rota_attn_desc(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("grid_t", ctypes.c_int32), ("grid_h", ctypes.c_int32),
                 ("grid_w", ctypes.c_int32), ("rope_dim", ctypes.c_int32 * 3),
                 ("had_block", ctypes.c_int32 * 3), ("rope_theta", ctypes.c_float),
-                ("sm_scale", ctypes.c_float), ("rope_phase", ctypes.c_float * 3)]
+                ("sm_scale", ctypes.c_float), ("rope_phase", ctypes.c_float * 3),
+                ("quant_block", ctypes.c_int32), ("max_group", ctypes.c_int32), ("row_sum", ctypes.c_int32)]
 
 
 class rota_attn_buffers(ctypes.Structure):
@@ -239,7 +240,8 @@ def default_had_block(d_a: int) -> int:
 
 def make_desc(B: int, H: int, head_dim: int, grid: Sequence[int], rope_dim: Sequence[int],
               had_block: Optional[Sequence[int]] = None, theta: float = 10000.0,
-              sm_scale: float = 0.0, rope_phase: Sequence[float] = (0.0, 0.0, 0.0)) -> rota_attn_desc:
+              sm_scale: float = 0.0, rope_phase: Sequence[float] = (0.0, 0.0, 0.0), quant_block: int = 64,
+              max_group: int = 64, row_sum: int = 0) -> rota_attn_desc:
     d = rota_attn_desc()
     d.B, d.H, d.head_dim = B, H, head_dim
     d.grid_t, d.grid_h, d.grid_w = grid
@@ -249,6 +251,7 @@ def make_desc(B: int, H: int, head_dim: int, grid: Sequence[int], rope_dim: Sequ
     d.rope_theta = theta
     d.sm_scale = sm_scale
     d.rope_phase[:] = [float(x) for x in rope_phase]
+    d.quant_block, d.max_group, d.row_sum = quant_block, max_group, row_sum
     return d
 
 

@@ -50,6 +50,9 @@ class Workload:
     # merged per-pair rotation angle added to every RoPE angle (0 = plain RoPE)
     had: Optional[Tuple[int, int, int]] = None
     rope_phase: Tuple[float, float, float] = (0.0, 0.0, 0.0)
+    # numerics options of the INT4 path: key group of the running max, row-sum reading
+    max_group: int = 64
+    row_sum: int = 0
 
     @property
     def N(self) -> int:
