@@ -72,15 +72,14 @@ struct Int4Params {
   int32_t* s_dump;
   uint8_t* p_dump;
   int dbg_r0, dbg_nr;
-  int row_sum;          // 0: l sums the codes; 1: l sums the unquantised 15 * 2^d
 };
 
 constexpr int kInt4Threads = 512;
 constexpr int kRowsPerCta = 2 * kBM;
 constexpr int kOps = 6;   // operand stages
 constexpr int kIssueRegs = 32;    // warps 0-3
-constexpr int kSoftmaxRegs = 136; // warps 4-11
-constexpr int kCorrRegs = 208;    // warps 12-15
+constexpr int kSoftmaxRegs = 128; // warps 4-11
+constexpr int kCorrRegs = 224;    // warps 12-15
 // Register split: the warpgroups' shares add up to the launch allocation
 // 512 * kLaunchRegs; the host refuses to launch a build whose register count
 // differs (setmaxnreg.inc would otherwise wait forever).
@@ -112,8 +111,8 @@ struct Int4Smem {
   static constexpr int SPILL_BYTES = G == 128 ? 2 * kBM * kBN * 4 : 0;
   static constexpr int OFF_BAR = OFF_SPILL + SPILL_BYTES;
   // barriers: op_full[OPS] op_empty[OPS] q_full s_full[2] s_empty[2]
-  //           p_full[2][2] p_empty[2][2] acc_full acc_empty l_full mma_done[2]
-  static constexpr int NBAR = 2 * OPS + 1 + 2 + 2 + 4 + 4 + 1 + 1 + 1 + 2;
+  //           p_full[2][2] p_empty[2][2] acc_full acc_empty l_full mma_done[2] turn[2]
+  static constexpr int NBAR = 2 * OPS + 1 + 2 + 2 + 4 + 4 + 1 + 1 + 1 + 2 + 2;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int BYTES = OFF_ABORT + 4;
@@ -157,12 +156,12 @@ __device__ __forceinline__ void setmaxnreg_issue() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 32;" ::: "memory");
 }
 __device__ __forceinline__ void setmaxnreg_softmax() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 136;" ::: "memory");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 128;" ::: "memory");
 }
 __device__ __forceinline__ void setmaxnreg_corr() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
 }
-static_assert(kIssueRegs == 32 && kSoftmaxRegs == 136 && kCorrRegs == 208, "setmaxnreg immediates");
+static_assert(kIssueRegs == 32 && kSoftmaxRegs == 128 && kCorrRegs == 224, "setmaxnreg immediates");
 
 // The max of one 64-key block's scores S = S_int * 2^-18 over the valid keys;
 // keys >= nvalid (MASK) are set to -inf in sr, so they never enter a max.
@@ -182,6 +181,25 @@ __device__ __forceinline__ float block_max(uint32_t (&sr)[kBN], int nvalid) {
     x3 = max3(x3, __uint_as_float(sr[k + 6]), __uint_as_float(sr[k + 7]));
   }
   return fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+}
+
+// Every code of one block by the exact function (the rare slow path of
+// block_codes); returns their sum.
+__device__ __noinline__ uint32_t block_codes_exact(const uint32_t* sr, int nvalid, float c18, float m, uint32_t* pw,
+                                                   const float* tau) {
+  uint32_t usum = 0;
+  for (int w = 0; w < kBN / 4; ++w) {
+    uint32_t word = 0;
+    for (int i = 0; i < 4; ++i) {
+      const int k = 4 * w + i;
+      const float d = k < nvalid ? __fmaf_rn(__uint_as_float(sr[k]), c18, -m) : -INFINITY;
+      const uint32_t u = pcode(d, tau);
+      word |= u << (8 * i);
+      usum += u;
+    }
+    pw[w] = word;
+  }
+  return usum;
 }
 
 // The P codes of one 64-key block of one softmax thread against the group
@@ -225,42 +243,32 @@ __device__ __forceinline__ uint32_t block_codes(const uint32_t (&sr)[kBN], int n
   uint32_t usum = sum_lo - 0xC0000000u;
   // Exact decisions (rare): some key of the warp's rows lies in the band
   // where the two roundings differ, or a row's max is so large that its max
-  // key could round past code 15.
+  // key could round past code 15.  Out of line, so that its registers do not
+  // weigh on the main path.
   const bool bad = (sum_lo != sum_hi) || !(fabsf(m) < kLogitBound);
   if (__any_sync(0xffffffffu, bad)) {
-    usum = 0;
+    // copies made only here, so the scores stay in registers on the main path
+    uint32_t s_copy[kBN], p_copy[kBN / 4];
 #pragma unroll
-    for (int w = 0; w < kBN / 4; ++w) {
-      uint32_t word = 0;
+    for (int k = 0; k < kBN; ++k) s_copy[k] = sr[k];
+    usum = block_codes_exact(s_copy, MASK ? nvalid : kBN, c18, m, p_copy, tau);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int k = 4 * w + i;
-        float d = __fmaf_rn(__uint_as_float(sr[k]), c18, -m);
-        if (MASK && k >= nvalid) d = -INFINITY;
-        const uint32_t u = pcode(d, tau);
-        word |= u << (8 * i);
-        usum += u;
-      }
-      pw[w] = word;
-    }
+    for (int w = 0; w < kBN / 4; ++w) pw[w] = p_copy[w];
   }
   return usum;
 }
 
-// The codes of one block with the row-sum reading chosen at run time; returns
-// the block's contribution to l (the code sum, or 15 sum 2^d).
-template <bool MASK>
+// The codes of one block; returns the block's contribution to l (the code
+// sum, or with R1 15 sum 2^d).
+template <bool MASK, bool R1>
 __device__ __forceinline__ float block_codes_l(const uint32_t (&sr)[kBN], int nvalid, float c18, float m,
-                                               uint32_t (&pw)[kBN / 4], const float* tau, bool r1) {
+                                               uint32_t (&pw)[kBN / 4], const float* tau) {
   float lsum = 0.f;
-  if (r1) {
-    block_codes<MASK, true>(sr, nvalid, c18, m, pw, tau, lsum);
-    return lsum;
-  }
-  return static_cast<float>(block_codes<MASK, false>(sr, nvalid, c18, m, pw, tau, lsum));
+  const uint32_t usum = block_codes<MASK, R1>(sr, nvalid, c18, m, pw, tau, lsum);
+  return R1 ? lsum : static_cast<float>(usum);
 }
 
-template <int D, int G>
+template <int D, int G, bool R1>
 __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid_constant__ Int4Params p) {
   using L = Int4Smem<D, G>;
   constexpr int kOps = L::OPS;
@@ -278,6 +286,9 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
   uint64_t* acc_empty = acc_full + 1;           // 4 correction warps hold ACC in registers
   uint64_t* l_full = acc_empty + 1;             // 8 softmax warps wrote their rows' l
   uint64_t* mma_done = l_full + 1;              // [2], one per issuing warp
+  // turn[t]: the other tile's 4 softmax warps finished a code phase, so tile
+  // t may take the exponential unit for its next one
+  uint64_t* turn = mma_done + 2;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + L::OFF_ABORT);
   float* sTau = reinterpret_cast<float*>(smem + L::OFF_TAU);
@@ -313,6 +324,8 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     mbar_init(l_full, 8);
     mbar_init(&mma_done[0], 1);
     mbar_init(&mma_done[1], 1);
+    mbar_init(&turn[0], 4);
+    mbar_init(&turn[1], 4);
     *sAbort = 0;
     fence_mbar_init();
   }
@@ -455,8 +468,8 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     }
     const float sq = row < npad ? __ldg(p.q_scale + head * p.nblk + row / kBN) : 0.f;
     const float* ksc = p.k_scale + head * p.nblk;
-    const bool dump_rows = p.s_dump != nullptr && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr;
-    const bool r1 = p.row_sum != 0;
+    const bool dumping = p.s_dump != nullptr;   // kernel argument: uniform
+    const bool dump_rows = dumping && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr;
 
     // S of block j -> registers; the buffer is released at once, so the MMA
     // computes the tile's next scores while these are coded
@@ -471,7 +484,7 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[t]);
-      if (__any_sync(0xffffffffu, dump_rows)) {
+      if (dumping) {
         const int nvalid = min(kBN, p.N - j * kBN);
 #pragma unroll
         for (int k = 0; k < kBN; ++k)
@@ -495,7 +508,7 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       sAlpha[(2 * t + sl) * kBM + r] = alpha;
       const bool moved = __any_sync(0xffffffffu, alpha != 1.f);
       if (lane == 0) sFlag[(2 * t + sl) * 4 + (warp & 3)] = moved ? 1 : 0;
-      if (__any_sync(0xffffffffu, dump_rows)) {
+      if (dumping) {
         const int nvalid = min(kBN, p.N - j * kBN);
 #pragma unroll
         for (int k = 0; k < kBN; ++k)
@@ -523,6 +536,22 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     // the key scales are read one block (pair) ahead
     float sk_next = __ldg(ksc), sk_next2 = nkb > 1 ? __ldg(ksc + 1) : 0.f;
 
+    // The two tiles take turns on the code phase (the exponentials): while
+    // one tile's warps code a block, the other tile's warps load, reduce and
+    // store theirs, so the exponential unit is not split between two phases
+    // in lockstep.  Tile 0 goes first.
+    int turns = 0;
+    auto my_turn = [&]() -> bool {
+      const bool ok = warp_wait(&turn[t], turns & 1, lim);
+      ++turns;
+      return ok;
+    };
+    auto pass_turn = [&]() {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&turn[t ^ 1]);
+    };
+    if (t == 1) pass_turn();
+
     float m = -INFINITY, l = 0.f;
     bool aborted = false;
     if constexpr (G == 64) {
@@ -536,8 +565,10 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         const float m_old = m;
         m = fmaxf(m, __fmul_rn(smax, c18));
         uint32_t pw[kBN / 4];
-        const float lsum = nvalid == kBN ? block_codes_l<false>(sr, nvalid, c18, m, pw, sTau, r1)
-                                         : block_codes_l<true>(sr, nvalid, c18, m, pw, sTau, r1);
+        if (!my_turn()) { aborted = true; break; }
+        const float lsum = nvalid == kBN ? block_codes_l<false, R1>(sr, nvalid, c18, m, pw, sTau)
+                                         : block_codes_l<true, R1>(sr, nvalid, c18, m, pw, sTau);
+        pass_turn();
         const float alpha = alpha_of(j == 0, m_old, m);
         l = __fmaf_rn(l, alpha, lsum);
         if (!emit(j, pw, alpha)) { aborted = true; break; }
@@ -574,9 +605,10 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         const float alpha = alpha_of(j0 == 0, m_old, m);
         uint32_t pw[kBN / 4];
         float lsum1 = 0.f;
+        if (!my_turn()) { aborted = true; break; }
         if (has1) {
-          lsum1 = nv1 == kBN ? block_codes_l<false>(sr, nv1, c1, m, pw, sTau, r1)
-                             : block_codes_l<true>(sr, nv1, c1, m, pw, sTau, r1);
+          lsum1 = nv1 == kBN ? block_codes_l<false, R1>(sr, nv1, c1, m, pw, sTau)
+                             : block_codes_l<true, R1>(sr, nv1, c1, m, pw, sTau);
           if (!emit(j1, pw, 1.f)) { aborted = true; break; }
         }
 #pragma unroll
@@ -587,8 +619,9 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
           sr[4 * i + 2] = __float_as_uint(x.z);
           sr[4 * i + 3] = __float_as_uint(x.w);
         }
-        const float lsum0 = nv0 == kBN ? block_codes_l<false>(sr, nv0, c0, m, pw, sTau, r1)
-                                       : block_codes_l<true>(sr, nv0, c0, m, pw, sTau, r1);
+        const float lsum0 = nv0 == kBN ? block_codes_l<false, R1>(sr, nv0, c0, m, pw, sTau)
+                                       : block_codes_l<true, R1>(sr, nv0, c0, m, pw, sTau);
+        pass_turn();
         l = __fadd_rn(__fmaf_rn(l, alpha, lsum0), lsum1);
         if (!emit(j0, pw, alpha)) { aborted = true; break; }
         if (warp_flag(sAbort)) { aborted = true; break; }
@@ -616,9 +649,8 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         if (!warp_wait(acc_full, u & 1, lim)) { aborted = true; break; }
         tc_fence_after();
         const uint32_t tO = tmem + L::T_O + t * kBM + t_lane;
-        // the block's ACC (all 128 query columns) and the first O chunk, in flight together
+        // the block's ACC, all 128 query columns
         uint32_t a[kBM];
-        uint32_t ob[2][32];
         {
           uint32_t(&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&a[0]);
           uint32_t(&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&a[32]);
@@ -628,10 +660,8 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
           tmem_ld32(tA + 32, a1);
           tmem_ld32(tA + 64, a2);
           tmem_ld32(tA + 96, a3);
-          if (j > 0) tmem_ld32(tO, ob[0]);
           tmem_wait_dep2(a0, a1);
           tmem_wait_dep2(a2, a3);
-          if (j > 0) tmem_wait_dep(ob[0]);
         }
         // ACC is in registers: the next P V may overwrite it
         tc_fence_before();
@@ -643,24 +673,30 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         const int* fl = sFlag + (2 * t + sl) * 4;
         const bool moved = j > 0 && (fl[0] | fl[1] | fl[2] | fl[3]) != 0;
         const float* al = sAlpha + (2 * t + sl) * kBM;
-        // O chunk cb + 1 is loaded while chunk cb is updated and stored
+        // O in two 64-column halves: one load round trip and two stores each
 #pragma unroll
-        for (int cb = 0; cb < kBM / 32; ++cb) {
-          uint32_t(&o)[32] = ob[cb & 1];
-          if (j > 0 && cb + 1 < kBM / 32) tmem_ld32(tO + 32 * (cb + 1), ob[(cb + 1) & 1]);
+        for (int hb = 0; hb < kBM / 64; ++hb) {
+          uint32_t o[64];
+          uint32_t(&o0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
+          uint32_t(&o1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[32]);
+          if (j > 0) {
+            tmem_ld32(tO + 64 * hb, o0);
+            tmem_ld32(tO + 64 * hb + 32, o1);
+            tmem_wait_dep2(o0, o1);
+          }
           if (j == 0) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(a[32 * cb + i]), s18));
+            for (int i = 0; i < 64; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(a[64 * hb + i]), s18));
           } else if (moved) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              const float4 a4 = *reinterpret_cast<const float4*>(al + 32 * cb + i);
+            for (int i = 0; i < 64; i += 4) {
+              const float4 a4 = *reinterpret_cast<const float4*>(al + 64 * hb + i);
               float x0, x1, x2, x3;
               // O alpha (one rounding), then + s ACC (one rounding)
               fma2(x0, x1, __uint_as_float(o[i]), __uint_as_float(o[i + 1]), a4.x, a4.y, 0.f, 0.f);
               fma2(x2, x3, __uint_as_float(o[i + 2]), __uint_as_float(o[i + 3]), a4.z, a4.w, 0.f, 0.f);
-              fma2(x0, x1, __uint_as_float(a[32 * cb + i]), __uint_as_float(a[32 * cb + i + 1]), s18, s18, x0, x1);
-              fma2(x2, x3, __uint_as_float(a[32 * cb + i + 2]), __uint_as_float(a[32 * cb + i + 3]), s18, s18, x2, x3);
+              fma2(x0, x1, __uint_as_float(a[64 * hb + i]), __uint_as_float(a[64 * hb + i + 1]), s18, s18, x0, x1);
+              fma2(x2, x3, __uint_as_float(a[64 * hb + i + 2]), __uint_as_float(a[64 * hb + i + 3]), s18, s18, x2, x3);
               o[i] = __float_as_uint(x0);
               o[i + 1] = __float_as_uint(x1);
               o[i + 2] = __float_as_uint(x2);
@@ -668,16 +704,16 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              float o0, o1;
-              fma2(o0, o1, __uint_as_float(a[32 * cb + i]), __uint_as_float(a[32 * cb + i + 1]), s18, s18,
+            for (int i = 0; i < 64; i += 2) {
+              float x0, x1;
+              fma2(x0, x1, __uint_as_float(a[64 * hb + i]), __uint_as_float(a[64 * hb + i + 1]), s18, s18,
                    __uint_as_float(o[i]), __uint_as_float(o[i + 1]));
-              o[i] = __float_as_uint(o0);
-              o[i + 1] = __float_as_uint(o1);
+              o[i] = __float_as_uint(x0);
+              o[i + 1] = __float_as_uint(x1);
             }
           }
-          tmem_st32(tO + 32 * cb, o);
-          if (j > 0 && cb + 1 < kBM / 32) tmem_wait_dep(ob[(cb + 1) & 1]);
+          tmem_st32(tO + 64 * hb, o0);
+          tmem_st32(tO + 64 * hb + 32, o1);
         }
         tmem_st_wait();
         // this tile's codes and alpha of block j are consumed

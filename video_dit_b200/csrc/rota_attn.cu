@@ -185,6 +185,16 @@ rota_status launch_int4_kernel(K kernel, int smem, dim3 grid, cudaStream_t s, co
   return cuda_status(cudaGetLastError());
 }
 
+// The INT4 kernel instantiation for a head dim, a max group and a row-sum reading.
+template <int D>
+rota_status launch_int4_variant(bool g128, bool r1, dim3 grid, cudaStream_t s, const rota::Int4Params& p) {
+  if (g128)
+    return r1 ? launch_int4_kernel(rota::attn_int4_kernel<D, 128, true>, rota::Int4Smem<D, 128>::ALLOC, grid, s, p)
+              : launch_int4_kernel(rota::attn_int4_kernel<D, 128, false>, rota::Int4Smem<D, 128>::ALLOC, grid, s, p);
+  return r1 ? launch_int4_kernel(rota::attn_int4_kernel<D, 64, true>, rota::Int4Smem<D, 64>::ALLOC, grid, s, p)
+            : launch_int4_kernel(rota::attn_int4_kernel<D, 64, false>, rota::Int4Smem<D, 64>::ALLOC, grid, s, p);
+}
+
 }  // namespace
 
 namespace {
@@ -405,7 +415,6 @@ static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers*
   p.N = d->N;
   p.nblk = npad_of(d->N) / 64;
   p.kappa = kappa_of(d);
-  p.row_sum = d->row_sum;
   std::memcpy(p.tau, tau_table().tau, sizeof(p.tau));
   {
     std::lock_guard<std::mutex> g(g_inject.mu);
@@ -453,13 +462,11 @@ static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers*
   // 2. attention
   const dim3 grid((d->N + rota::kRowsPerCta - 1) / rota::kRowsPerCta, p.nheads, batches);
   // the debug dump runs the same kernel with its dump pointers set
-  const bool g128 = d->max_group == 128;
+  const bool g128 = d->max_group == 128, r1 = d->row_sum != 0;
   if (d->head_dim == 128)
-    st = g128 ? launch_int4_kernel(rota::attn_int4_kernel<128, 128>, rota::Int4Smem<128, 128>::ALLOC, grid, s, p)
-              : launch_int4_kernel(rota::attn_int4_kernel<128, 64>, rota::Int4Smem<128, 64>::ALLOC, grid, s, p);
+    st = launch_int4_variant<128>(g128, r1, grid, s, p);
   else
-    st = g128 ? launch_int4_kernel(rota::attn_int4_kernel<64, 128>, rota::Int4Smem<64, 128>::ALLOC, grid, s, p)
-              : launch_int4_kernel(rota::attn_int4_kernel<64, 64>, rota::Int4Smem<64, 64>::ALLOC, grid, s, p);
+    st = launch_int4_variant<64>(g128, r1, grid, s, p);
   return st;
 }
 
