@@ -193,6 +193,67 @@ def accuracy_sample(w, q, k, v, out, h, rows):
             "tolerance_max_abs": 2e-3}
 
 
+def run_qkv_fused(args, w):
+    """--qkv-fused C: the QKV projection (x [B,N,C] @ W^T, W [3 H d, C], fp16)
+    followed by the prologue, two ways on one GPU: the fused call
+    (rota_attn_qkv_prepare: Q, K, V never leave the chip) and a cuBLAS fp16
+    GEMM (torch.matmul) writing Q, K, V to HBM, then rota_attn_prepare_qk.
+    CUDA events around each, W warm-up steps then K timed ones."""
+    import torch
+    from video_dit_b200 import rota_attn as ra
+    C = args.qkv_fused
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev).manual_seed(0)
+    x = torch.randn((w.B, w.N, C), generator=g, device=dev, dtype=torch.float32).to(torch.float16)
+    wt = (torch.randn((3 * w.H * w.d, C), generator=g, device=dev, dtype=torch.float32) / C ** 0.5).to(torch.float16)
+    desc = ra.make_desc(w.B, w.H, w.d, w.grid, w.rope_dim, w.had_block, w.theta, rope_phase=w.rope_phase,
+                        max_group=w.max_group, row_sum=w.row_sum)
+    att = ra.RotaAttention(desc, device=dev, need_fp16=False)
+    stream = torch.cuda.current_stream(dev)
+
+    def fused():
+        ra._check(ra.rota_attn_qkv_prepare(desc, x, wt, C, None, att.buffers), "qkv_prepare")
+
+    def unfused():
+        qkv = torch.matmul(x, wt.t())                                   # [B, N, 3 H d] fp16 (cuBLAS)
+        qkv = qkv.view(w.B, w.N, 3, w.H, w.d).permute(2, 0, 3, 1, 4).contiguous()  # [3, B, H, N, d]
+        att.prepare(qkv[0], qkv[1], qkv[2])
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    ms_fused = timed(fused)
+    st = ra.rota_attn_get_error()
+    if st != ra.ROTA_OK:
+        raise RuntimeError(f"device error: {ra.rota_attn_status_string(st)}")
+    ms_unfused = timed(unfused)
+    flops = 2.0 * w.B * w.N * C * 3 * w.H * w.d
+    qkv_bytes = 3 * w.B * w.H * w.N * w.d * 2
+    nblk = (w.N + 63) // 64
+    code_bytes = w.B * w.H * (3 * nblk * 64 * w.d // 2 + 2 * nblk * 4 + nblk * w.d * 4)
+    in_bytes = x.numel() * 2 + wt.numel() * 2
+    line = {"metric": "QKV projection + prologue, fused vs cuBLAS GEMM + prologue", "unit": "ms",
+            "value": ms_fused, "higher_is_better": False, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "dtype": "fp16 x, W; fp32 accumulation; s4 codes",
+            "config": {"workload": f"{w.name} (B={w.B} H={w.H} N={w.N} d={w.d}) with C={C}", "C": C},
+            "fused_ms": ms_fused, "unfused_ms": ms_unfused, "gemm_tflops_fused": flops / (ms_fused * 1e-3) / 1e12,
+            "algorithmic_bytes": {"inputs_x_w": in_bytes, "qkv_fp16_round_trip_avoided": 2 * qkv_bytes,
+                                  "codes_and_scales_written": code_bytes,
+                                  "fused_total": in_bytes + code_bytes,
+                                  "unfused_total": in_bytes + 2 * qkv_bytes + code_bytes}}
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args, w, world, rank):
     """--impl reference: the CPU oracle as it stands, on bounded samples."""
     if rank != 0:
@@ -235,6 +296,7 @@ def main():
     ap.add_argument("--chunk-heads", type=int, default=0)     # heads per chunk of the e2e pipeline (0: library default)
     ap.add_argument("--no-e2e", action="store_true")          # skip the end-to-end loop (profiling runs)
     ap.add_argument("--accuracy-rows", type=int, default=32)  # sampled rows of the accuracy record (0: none)
+    ap.add_argument("--qkv-fused", type=int, default=0)       # C > 0: time the fused QKV projection + prologue
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -244,6 +306,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, w, world, rank)
+        return
+    if args.qkv_fused:
+        run_qkv_fused(args, w)
         return
 
     import torch

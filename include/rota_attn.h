@@ -182,6 +182,32 @@ rota_status rota_attn_prepare_qk(const rota_attn_desc* desc, const uint16_t* q, 
                                  const rota_attn_buffers* buf, void* stream);
 
 /*
+ * The QKV projection of the DiT block with the prologue fused into its
+ * epilogue (the abstract places the INT4 attention inside the DiT block, right
+ * after this projection): fp16 Q, K, V are computed and quantised on chip and
+ * never written to HBM.  Same results as the projection followed by
+ * rota_attn_prepare_qk on its fp16 outputs.
+ *   x    : fp16 [B, N, C] device, the block's input tokens (16-byte aligned)
+ *   w    : fp16 [3 * H * head_dim, C] device, the projection weights: rows
+ *          h*head_dim .. +head_dim-1 give Q of head h, rows H*head_dim + ...
+ *          K, rows 2*H*head_dim + ... V (16-byte aligned)
+ *   C    : input channels, a multiple of 64 (at most 2^20)
+ *   q = x W_q^T, k = x W_k^T, v = x W_v^T per head with fp32 accumulation,
+ *   each rounded to fp16; then, per head, exactly rota_attn_prepare_qk's
+ *   prologue (codes and scales of INT4 heads; q_rope / k_rope of flagged
+ *   heads).
+ *   head_flags, buf: as for rota_attn_prepare_qk.
+ *   v_out: fp16 [B, H, N, head_dim] device; the fp16 V of the flagged heads is
+ *          written there (the FP16 fallback's v); may be NULL when no head is
+ *          flagged.
+ * ROTA_ERR_INVALID_ARG for a null / misaligned pointer or C not a positive
+ * multiple of 64.
+ */
+rota_status rota_attn_qkv_prepare(const rota_attn_desc* desc, const uint16_t* x, const uint16_t* w, int32_t C,
+                                  const uint8_t* head_flags, const rota_attn_buffers* buf, uint16_t* v_out,
+                                  void* stream);
+
+/*
  * INT4 attention (the abstract's mixed-precision INT4 FlashAttention) for the
  * heads whose flag is 0.  Exact integer Q K^T on the tensor cores (the codes
  * as exact e4m3 values, fp32 accumulation that stays integral); scores

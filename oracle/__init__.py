@@ -71,6 +71,8 @@ def lib():
         L.oracle_pcode.restype = i32
         L.oracle_pcode_array.argtypes = [P, P, i64, P]
         L.oracle_pcode_array.restype = None
+        L.oracle_qkv_project.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P]
+        L.oracle_qkv_project.restype = None
         L.oracle_attn_int4.argtypes = [i32, i32, i32, i32, f32, i32, i32] + [P] * 6 + \
             [i32, i32, i32, i32, i32, P, P, P]
         L.oracle_attn_int4.restype = i32
@@ -218,6 +220,19 @@ def prepare(q, k, v, grid, rope_dim, had_block, theta=10000.0, flags=None, phase
     if rc != 0:
         raise MemoryError("oracle_prepare failed")
     return out
+
+
+def qkv_project(x, w, H: int, D: int):
+    """The QKV projection in front of the path: x fp16 [B, N, C], w fp16
+    [3 H D, C] -> fp16 q, k, v [B, H, N, D] (exact sums, rounded to fp32 and
+    then to fp16)."""
+    x, w = _h(x), _h(w)
+    B, N, C = x.shape
+    q = np.zeros((B, H, N, D), np.uint16)
+    k = np.zeros_like(q)
+    v = np.zeros_like(q)
+    lib().oracle_qkv_project(B, N, C, H, D, _p(x), _p(w), _p(q), _p(k), _p(v))
+    return q.view(np.float16), k.view(np.float16), v.view(np.float16)
 
 
 def attn_int4(prep: dict, N: int, sm_scale: float, b: int, h: int, r0: int, nr: int,

@@ -469,6 +469,41 @@ int oracle_prepare(int B, int H, int N, int d, const int grid[3], const int rope
 }
 
 /* ----------------------------------------------------------------------- */
+/* The QKV projection in front of the path (the abstract places the INT4    */
+/* attention inside the DiT block, right after it): per head h and token n, */
+/* q[b,h,n,c] = sum_k x[b,n,k] w[h*D + c, k], k[...] with rows H*D + h*D + c,*/
+/* v[...] with rows 2*H*D + h*D + c; each sum accumulated exactly (double:   */
+/* the fp16 products are exact, and the sums of the pinned inputs too),     */
+/* rounded to fp32 (reading: an fp32 accumulation whose order the pages do  */
+/* not fix, taken as the correctly rounded fp32 value of the sum) and then  */
+/* to fp16 -- the fp16 Q, K, V the prologue takes.  x [B,N,C], w [3HD,C],   */
+/* outputs fp16 bit patterns [B,H,N,D].                                      */
+/* ----------------------------------------------------------------------- */
+
+void oracle_qkv_project(int B, int N, int C, int H, int D, const uint16_t *x, const uint16_t *w,
+                        uint16_t *q, uint16_t *k, uint16_t *v)
+{
+    uint16_t *outs[3] = {q, k, v};
+    double *xrow = (double *)malloc(sizeof(double) * (size_t)C);
+    double *wrow = (double *)malloc(sizeof(double) * (size_t)C);
+    if (!xrow || !wrow) { free(xrow); free(wrow); return; }
+    for (int m = 0; m < 3; ++m)
+        for (int h = 0; h < H; ++h)
+            for (int c = 0; c < D; ++c) {
+                const uint16_t *wr = w + ((long)(m * H + h) * D + c) * C;
+                for (int kk = 0; kk < C; ++kk) wrow[kk] = (double)oracle_half_to_float(wr[kk]);
+                for (int b = 0; b < B; ++b)
+                    for (int n = 0; n < N; ++n) {
+                        const uint16_t *xr = x + ((long)b * N + n) * C;
+                        double acc = 0.0;
+                        for (int kk = 0; kk < C; ++kk) acc += (double)oracle_half_to_float(xr[kk]) * wrow[kk];
+                        outs[m][(((long)b * H + h) * N + n) * D + c] = oracle_float_to_half((float)acc);
+                    }
+            }
+    free(xrow); free(wrow);
+}
+
+/* ----------------------------------------------------------------------- */
 /* Step 5: range-optimised P code of one exponent d (fp32, d <= ~0).        */
 /* P = 2^d in (0,1] is mapped to the unsigned code u = RNE(15 P) with the   */
 /* fixed scale 1/15 and zero-point 0, in exact real arithmetic on the fp32  */

@@ -626,3 +626,27 @@ def test_max_group_128_closed_form():
     # R1 with 128-key groups: 15 * 2^-1 = 7.5 per block-0 key and per other block-1 key
     o128r1 = oracle.attn_int4(prep, 128, sm, 0, 0, 0, 1, group=128, rowsum=1)
     assert np.abs(o128r1[0] - num128 / (64 * 7.5 + 15 + 63 * 7.5)).max() < 1e-14
+
+
+# ------------------------------------------------------------- QKV projection
+
+def test_qkv_project_matches_numpy_and_exact_grid():
+    """The oracle's projection against numpy (float64 matmul -> fp32 -> fp16)
+    on general fp16 inputs, and against exact integer arithmetic on the grid
+    inputs (k / 16 times j / 64: sums of multiples of 2^-10)."""
+    w = synth.scaled(synth.WORKLOADS["wan480"], "qkv_pin", H=2, grid=(1, 3, 7))      # N = 21
+    C = 128
+    for exact in (False, True):
+        x, wt = synth.make_qkv_inputs(w, C, seed=5, exact=exact)
+        q, k, v = oracle.qkv_project(x, wt, w.H, w.d)
+        full = x[0].astype(np.float64) @ wt.astype(np.float64).T                    # [N, 3 H d]
+        want = full.astype(np.float32).astype(np.float16)
+        for m, out in enumerate((q, k, v)):
+            for h in range(w.H):
+                cols = want[:, (m * w.H + h) * w.d:(m * w.H + h + 1) * w.d]
+                assert np.array_equal(out[0, h].view(np.uint16), cols.view(np.uint16)), (exact, m, h)
+        if exact:
+            xi = np.round(x[0].astype(np.float64) * 16).astype(np.int64)
+            wi = np.round(wt.astype(np.float64) * 64).astype(np.int64)
+            ints = xi @ wi.T                                                           # exact, units 2^-10
+            assert np.array_equal(ints.astype(np.float64) / 1024.0, full)

@@ -214,10 +214,18 @@ __device__ __forceinline__ uint32_t pack8_f(float4 a, float4 b, float inv) {
          ((code_nibble(a.w, inv) | (code_nibble(b.w, inv) << 4)) << 24);
 }
 
+// 16 bytes of an fp16 tile row: read-only global loads, or plain loads from
+// a shared-memory tile (the QKV-projection epilogue).
+template <bool SMEM>
+__device__ __forceinline__ uint4 load16(const __half* p) {
+  if (SMEM) return *reinterpret_cast<const uint4*>(p);
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
 // fp16 tile [64, D] of one (head, block) -> fp32 smem rows of stride D + 4
 // (16-byte aligned rows).  Every thread issues all of its 16-byte loads before
 // it converts any, so a CTA waits for one memory latency rather than one per load.
-template <int D>
+template <int D, bool SMEM>
 __device__ __forceinline__ void load_tile(const __half* src, int n0, int N, float* X) {
   constexpr int LD = D + 4;
   constexpr int PER = 64 * D / 8 / kPrologueThreads;
@@ -228,7 +236,7 @@ __device__ __forceinline__ void load_tile(const __half* src, int n0, int N, floa
     const int i = threadIdx.x + k * kPrologueThreads;
     const int r = i / (D / 8), ch = i % (D / 8);
     const int n = n0 + r;
-    u[k] = n < N ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)n * D + ch * 8)) : make_uint4(0, 0, 0, 0);
+    u[k] = n < N ? load16<SMEM>(src + (size_t)n * D + ch * 8) : make_uint4(0, 0, 0, 0);
   }
 #pragma unroll
   for (int k = 0; k < PER; ++k) {
@@ -243,22 +251,21 @@ __device__ __forceinline__ void load_tile(const __half* src, int n0, int N, floa
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const __grid_constant__ PrologueParams p) {
+// The prologue of one (64-token block blk, head (b, h), tensor which = Q / K
+// / V), by all kPrologueThreads threads of the block.  src: the tensor's rows
+// of this head, token n at src + n * D (SMEM: a shared-memory tile holding
+// rows n0 .. n0 + 63, addressed the same way).  X, red, sPos: shared scratch.
+// Not for a flagged head's V (the caller keeps the fp16 V itself).
+template <int D, bool SMEM>
+__device__ __forceinline__ void prologue_job(const PrologueParams& p, const __half* src, int blk, int h, int b,
+                                             int which, float* X, float* red, int4* sPos) {
   constexpr int LD = D + 4;
-  __shared__ __align__(16) float X[64 * LD];
-  __shared__ float red[kPrologueThreads / 32];
-  __shared__ int4 sPos[64];
-
-  const int blk = blockIdx.x, h = blockIdx.y;
-  const int b = blockIdx.z / 3, which = blockIdx.z % 3;
   const size_t head = (size_t)b * p.H + h;
   const int n0 = blk * 64;
   const bool flagged = head_flagged(p, h);
   const int npad = p.nblk * 64;
 
   if (which < 2) {
-    const __half* src = (which == 0 ? p.q : p.k) + head * p.N * D;
     if (flagged) {
       // FP16 fallback head: RoPE only, stored as fp16 for the fallback kernel.
       __half* dst = (which == 0 ? p.q_rope : p.k_rope) + head * p.N * D;
@@ -268,7 +275,7 @@ __global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const __g
         if (n >= p.N) continue;
         int pos[3];
         token_pos(p, n, pos);
-        uint4 u = __ldg(reinterpret_cast<const uint4*>(src + (size_t)n * D + ch * 8));
+        uint4 u = load16<SMEM>(src + (size_t)n * D + ch * 8);
         __half2* h2 = reinterpret_cast<__half2*>(&u);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -296,7 +303,7 @@ __global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const __g
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
       const int n = n0 + rb + k * RSTEP;
-      u[k] = n < p.N ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)n * D + ch * 8)) : make_uint4(0, 0, 0, 0);
+      u[k] = n < p.N ? load16<SMEM>(src + (size_t)n * D + ch * 8) : make_uint4(0, 0, 0, 0);
     }
     // token coordinates of the block's tokens, while the loads are in flight
     if (threadIdx.x < 64) {
@@ -425,7 +432,7 @@ __global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const __g
 
   // V: per (block, channel) scale, no RoPE, no rotation.
   if (flagged) return;
-  load_tile<D>(p.v + head * p.N * D, n0, p.N, X);
+  load_tile<D, SMEM>(src, n0, p.N, X);
   __syncthreads();
   // kPrologueThreads / D neighbouring lanes share a channel, each taking 64 / TPC rows
   constexpr int TPC = kPrologueThreads / D;
@@ -459,6 +466,18 @@ __global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const __g
       *reinterpret_cast<uint4*>(dst + j) = make_uint4(w[j], w[j + 1], w[j + 2], w[j + 3]);
     if (part == 0) p.v_scale[(head * p.nblk + blk) * D + c] = scale;
   }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const __grid_constant__ PrologueParams p) {
+  constexpr int LD = D + 4;
+  __shared__ __align__(16) float X[64 * LD];
+  __shared__ float red[kPrologueThreads / 32];
+  __shared__ int4 sPos[64];
+  const int h = blockIdx.y, b = blockIdx.z / 3, which = blockIdx.z % 3;
+  const size_t head = (size_t)b * p.H + h;
+  const __half* src = (which == 0 ? p.q : which == 1 ? p.k : p.v) + head * p.N * D;
+  prologue_job<D, false>(p, src, blockIdx.x, h, b, which, X, red, sPos);
 }
 
 }  // namespace rota

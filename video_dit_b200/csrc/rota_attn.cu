@@ -19,6 +19,7 @@
 #include "calib.cuh"
 #include "attn_int4.cuh"
 #include "prologue.cuh"
+#include "qkv_prologue.cuh"
 
 namespace {
 
@@ -155,6 +156,44 @@ bool int4_buffers_ok(const rota_attn_buffers* buf, bool with_work) {
     if (!ptr || !aligned16(ptr)) return false;
   if (!buf->q_scale || !buf->k_scale || !aligned4(buf->q_scale) || !aligned4(buf->k_scale)) return false;
   return !with_work || (buf->int4_work && aligned16(buf->int4_work));
+}
+
+// The prologue's parameters for a descriptor, flags and buffers (the input
+// pointers q, k, v are left to the caller).
+void fill_prologue_params(const rota_attn_desc* d, const uint8_t* head_flags, const rota_attn_buffers* buf,
+                          rota::PrologueParams* pp) {
+  rota::PrologueParams& p = *pp;
+  p.q_codes = buf->q_codes;
+  p.k_codes = buf->k_codes;
+  p.q_scale = buf->q_scale;
+  p.k_scale = buf->k_scale;
+  p.v_codes = buf->v_codes;
+  p.v_scale = buf->v_scale;
+  p.q_rope = reinterpret_cast<__half*>(buf->q_rope);
+  p.k_rope = reinterpret_cast<__half*>(buf->k_rope);
+  p.cos_tab = buf->rope_cos;
+  p.sin_tab = buf->rope_sin;
+  p.H = d->H;
+  p.N = d->N;
+  p.nblk = npad_of(d->N) / 64;
+  p.grid_h = d->grid_h;
+  p.grid_w = d->grid_w;
+  const int extent[3] = {d->grid_t, d->grid_h, d->grid_w};
+  int coff = 0, toff = 0;
+  for (int a = 0; a < 3; ++a) {
+    p.rope_dim[a] = d->rope_dim[a];
+    p.had[a] = d->had_block[a];
+    p.coff[a] = coff;
+    p.toff[a] = toff;
+    p.rnorm[a] = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d->had_block[a])));
+    p.fused[a] = d->had_block[a] <= 1 || (d->had_block[a] <= 8 && coff % d->had_block[a] == 0);
+    p.dense[a] = hadamard_rows(d->had_block[a], p.hneg[a]) ? 1 : 0;
+    if (!p.fused[a]) p.any_unfused = 1;
+    coff += d->rope_dim[a];
+    toff += extent[a] * (d->rope_dim[a] / 2);
+  }
+  for (int h = 0; h < d->H; ++h)
+    if (head_flags && head_flags[h]) p.flags[h >> 5] |= 1u << (h & 31);
 }
 
 // Heads with flag == want, written to `heads`; returns their count.
@@ -346,41 +385,10 @@ rota_status rota_attn_prepare_qk(const rota_attn_desc* d, const uint16_t* q, con
     return ROTA_ERR_INVALID_ARG;
 
   rota::PrologueParams p{};
+  fill_prologue_params(d, head_flags, buf, &p);
   p.q = reinterpret_cast<const __half*>(q);
   p.k = reinterpret_cast<const __half*>(k);
   p.v = reinterpret_cast<const __half*>(v);
-  p.q_codes = buf->q_codes;
-  p.k_codes = buf->k_codes;
-  p.q_scale = buf->q_scale;
-  p.k_scale = buf->k_scale;
-  p.v_codes = buf->v_codes;
-  p.v_scale = buf->v_scale;
-  p.q_rope = reinterpret_cast<__half*>(buf->q_rope);
-  p.k_rope = reinterpret_cast<__half*>(buf->k_rope);
-  p.cos_tab = buf->rope_cos;
-  p.sin_tab = buf->rope_sin;
-  p.H = d->H;
-  p.N = d->N;
-  p.nblk = npad_of(d->N) / 64;
-  p.grid_h = d->grid_h;
-  p.grid_w = d->grid_w;
-  const int extent[3] = {d->grid_t, d->grid_h, d->grid_w};
-  int coff = 0, toff = 0;
-  for (int a = 0; a < 3; ++a) {
-    p.rope_dim[a] = d->rope_dim[a];
-    p.had[a] = d->had_block[a];
-    p.coff[a] = coff;
-    p.toff[a] = toff;
-    p.rnorm[a] = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d->had_block[a])));
-    p.fused[a] = d->had_block[a] <= 1 || (d->had_block[a] <= 8 && coff % d->had_block[a] == 0);
-    p.dense[a] = hadamard_rows(d->had_block[a], p.hneg[a]) ? 1 : 0;
-    if (!p.fused[a]) p.any_unfused = 1;
-    coff += d->rope_dim[a];
-    toff += extent[a] * (d->rope_dim[a] / 2);
-  }
-  for (int h = 0; h < d->H; ++h)
-    if (head_flags && head_flags[h]) p.flags[h >> 5] |= 1u << (h & 31);
-
   const dim3 grid(p.nblk, d->H, d->B * 3);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d->head_dim == 128)
@@ -391,6 +399,45 @@ rota_status rota_attn_prepare_qk(const rota_attn_desc* d, const uint16_t* q, con
 }
 
 // part: 1 = widen only, 2 = attention only, 3 = both
+rota_status rota_attn_qkv_prepare(const rota_attn_desc* d, const uint16_t* x, const uint16_t* w, int32_t C,
+                                  const uint8_t* head_flags, const rota_attn_buffers* buf, uint16_t* v_out,
+                                  void* stream) {
+  rota_status st = rota_attn_validate(d);
+  if (st != ROTA_OK) return st;
+  if (!buf || !x || !w || !buf->rope_cos || !buf->rope_sin) return ROTA_ERR_INVALID_ARG;
+  if (C < 64 || C % 64 != 0 || !aligned16(x) || !aligned16(w)) return ROTA_ERR_INVALID_ARG;
+  if (static_cast<long long>(C) > (1ll << 20)) return ROTA_ERR_UNSUPPORTED;
+  int16_t tmp[256];
+  const int n_int4 = select_heads(d, head_flags, 0, tmp);
+  const int n_fp16 = d->H - n_int4;
+  if (n_int4 > 0 && !int4_buffers_ok(buf, false)) return ROTA_ERR_INVALID_ARG;
+  if (n_fp16 > 0 && (!buf->q_rope || !buf->k_rope || !v_out || !aligned16(buf->q_rope) || !aligned16(buf->k_rope) ||
+                     !aligned16(v_out)))
+    return ROTA_ERR_INVALID_ARG;
+  static rota::QkvParams p;   // large (tensor maps, prologue tables); filled under a lock
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  p = rota::QkvParams{};
+  fill_prologue_params(d, head_flags, buf, &p.pro);
+  p.v_out = reinterpret_cast<__half*>(v_out);
+  p.C = C;
+  p.timeout_ns = kDefaultTimeoutNs;
+  const int D = d->head_dim;
+  if ((st = make_fp16_map(&p.tm_x, x, static_cast<uint64_t>(d->B) * d->N, C, 128)) != ROTA_OK) return st;
+  if ((st = make_fp16_map(&p.tm_w, w, static_cast<uint64_t>(3) * d->H * D, C, static_cast<uint32_t>(D))) != ROTA_OK)
+    return st;
+  const dim3 grid((d->N + 127) / 128, d->H, d->B);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (D == 128) {
+    if ((st = set_smem(rota::qkv_prologue_kernel<128>, rota::QkvSmem<128>::ALLOC)) != ROTA_OK) return st;
+    rota::qkv_prologue_kernel<128><<<grid, rota::kQkvThreads, rota::QkvSmem<128>::ALLOC, s>>>(p);
+  } else {
+    if ((st = set_smem(rota::qkv_prologue_kernel<64>, rota::QkvSmem<64>::ALLOC)) != ROTA_OK) return st;
+    rota::qkv_prologue_kernel<64><<<grid, rota::kQkvThreads, rota::QkvSmem<64>::ALLOC, s>>>(p);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
 static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers* buf, const uint8_t* head_flags,
                                float* out, void* stream, bool dump, int b, int h, int r0, int nr, int32_t* s_out,
                                uint8_t* p_out, int part = 3) {

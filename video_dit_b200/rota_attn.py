@@ -55,6 +55,7 @@ _SIGS = {
     "rota_attn_build_rope_tables": ([_D, _P, _P], ctypes.c_int),
     "rota_attn_prepare_qk": ([_D, _P, _P, _P, _P, _BUF, _P], ctypes.c_int),
     "rota_attn_fwd_int4": ([_D, _BUF, _P, _P, _P], ctypes.c_int),
+    "rota_attn_qkv_prepare": ([_D, _P, _P, ctypes.c_int32, _P, _BUF, _P, _P], ctypes.c_int),
     "rota_attn_int4_widen": ([_D, _BUF, _P, _P], ctypes.c_int),
     "rota_attn_int4_attend": ([_D, _BUF, _P, _P, _P], ctypes.c_int),
     "rota_attn_fwd_fp16_fallback": ([_D, _BUF, _P, _P, _P, _P], ctypes.c_int),
@@ -145,6 +146,12 @@ def rota_attn_prepare_qk(desc, q, k, v, head_flags, buffers: rota_attn_buffers, 
 def rota_attn_fwd_int4(desc, buffers: rota_attn_buffers, head_flags, out, stream=None) -> int:
     return _lib.rota_attn_fwd_int4(ctypes.byref(desc), ctypes.byref(buffers), _flags(head_flags), _ptr(out),
                                    _stream(stream))
+
+
+def rota_attn_qkv_prepare(desc, x, w, C: int, head_flags, buffers: rota_attn_buffers, v_out=None,
+                          stream=None) -> int:
+    return _lib.rota_attn_qkv_prepare(ctypes.byref(desc), _ptr(x), _ptr(w), int(C), _flags(head_flags),
+                                      ctypes.byref(buffers), _ptr(v_out), _stream(stream))
 
 
 def rota_attn_int4_widen(desc, buffers: rota_attn_buffers, head_flags, stream=None) -> int:

@@ -140,3 +140,35 @@ def make_inputs(w: Workload, seed: int = 0):
             v[:, h, tok, :] *= w.v_token_scale
     return (q.to(torch.float16).numpy(), k.to(torch.float16).numpy(),
             v.to(torch.float16).numpy())
+
+
+def make_qkv_inputs(w: Workload, C: int, seed: int = 0, exact: bool = True):
+    """Inputs of the fused QKV projection: x fp16 [B, N, C] and the projection
+    weights fp16 [3 H d, C] (rows of head h: Q at h d, K at H d + h d, V at
+    2 H d + h d), Gaussian so that q, k, v come out about N(0, 1); the Q / K
+    rows of the workload's outlier channels are scaled by its qk_scale.
+    exact=True puts x on the grid k / 16 (|k| <= 128) and W on j / 64, so every
+    product is a multiple of 2^-10 and every sum below 2^24 of those units:
+    the fp32 accumulation is then exact in any order, and a projection's
+    result does not depend on how it sums."""
+    B, H, N, d = w.B, w.H, w.N, w.d
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn((B, N, C), generator=g, dtype=torch.float64)
+    wt = torch.randn((3 * H * d, C), generator=g, dtype=torch.float64) / math.sqrt(C)
+    if any(w.qk_outliers):
+        g1 = torch.Generator().manual_seed(seed + 1)
+        off = 0
+        for a in range(3):
+            for h in range(H):
+                for m in (0, 1):
+                    perm = torch.randperm(w.rope_dim[a], generator=g1)
+                    rows = m * H * d + h * d + off + perm[: w.qk_outliers[a]]
+                    wt[rows] *= w.qk_scale
+            off += w.rope_dim[a]
+    if exact:
+        x = torch.clamp(torch.round(x * 16), -128, 128) / 16
+        wt = torch.round(wt * 64) / 64
+        assert float(wt.abs().max()) * 64 <= 2048
+        bound = C * 128 * float(wt.abs().max() * 64)          # |sum| in units of 2^-10
+        assert bound < 2 ** 24, "inputs too wide for an exact fp32 accumulation"
+    return x.to(torch.float16).numpy(), wt.to(torch.float16).numpy()
