@@ -254,6 +254,36 @@ def run_qkv_fused(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_mma_rates(args):
+    """--mma-rates: cycles per tcgen05.mma (M = 128, a chain of 4 x 256 MMAs
+    into one accumulator, operands in shared memory) for kind::f8f6f4 (e4m3),
+    kind::i8 (s8) and kind::f16 at N = 64, 128 and 256: the measurement the
+    choice of the Q K^T kind rests on."""
+    import torch
+    from video_dit_b200 import rota_attn as ra
+    torch.cuda.set_device(0)
+    cyc = torch.zeros(1, dtype=torch.int64, device="cuda")
+    names = {0: "f8f6f4 e4m3 x e4m3 -> f32", 1: "i8 s8 x s8 -> s32", 2: "f16 x f16 -> f32"}
+    iters, rows = 256, []
+    for kind in (0, 1, 2):
+        for n in (64, 128, 256):
+            best = None
+            for _ in range(max(1, args.steps)):
+                ra._check(ra.rota_attn_debug_mma_cycles(kind, n, iters, cyc), "mma_cycles")
+                torch.cuda.synchronize()
+                per = int(cyc.item()) / (4 * iters)
+                best = per if best is None else min(best, per)
+            kbytes = 32                                     # 32 bytes of K per operand row per MMA
+            k = kbytes if kind < 2 else kbytes // 2
+            rows.append({"kind": names[kind], "M": 128, "N": n, "K": k, "cycles_per_mma": best,
+                         "ops_per_cycle_per_sm": 2 * 128 * n * k / best})
+    st = ra.rota_attn_get_error()
+    if st != ra.ROTA_OK:
+        raise RuntimeError(f"device error: {ra.rota_attn_status_string(st)}")
+    print(json.dumps({"metric": "tcgen05.mma cycles per instruction (one CTA, dependent accumulation chain)",
+                      "unit": "cycles", "rates": rows}), flush=True)
+
+
 def run_reference(args, w, world, rank):
     """--impl reference: the CPU oracle as it stands, on bounded samples."""
     if rank != 0:
@@ -297,6 +327,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")          # skip the end-to-end loop (profiling runs)
     ap.add_argument("--accuracy-rows", type=int, default=32)  # sampled rows of the accuracy record (0: none)
     ap.add_argument("--qkv-fused", type=int, default=0)       # C > 0: time the fused QKV projection + prologue
+    ap.add_argument("--mma-rates", action="store_true")       # time tcgen05.mma per operand kind and shape
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -309,6 +340,9 @@ def main():
         return
     if args.qkv_fused:
         run_qkv_fused(args, w)
+        return
+    if args.mma_rates:
+        run_mma_rates(args)
         return
 
     import torch

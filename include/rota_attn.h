@@ -400,6 +400,18 @@ rota_status rota_attn_debug_pcode(const float* d, uint8_t* u, int64_t n, void* s
  * exits with ROTA_ERR_TIMEOUT.  One-shot; 0 disarms. */
 rota_status rota_attn_debug_inject_timeout(int32_t arm, uint64_t timeout_ns);
 
+/* Measurement of the tensor-core operand kinds the INT4 kernel chooses between
+ * for Q K^T (the abstract's INT4 FlashAttention: an exact integer product).
+ * One CTA issues `iters` x 4 tcgen05.mma of M = 128, N = n, 128 bytes of K per
+ * operand row per 4 MMAs, back to back into one TMEM accumulator, operands in
+ * shared memory.  kind: 0 = f8f6f4 (e4m3 x e4m3 -> f32), 1 = i8 (s8 x s8 ->
+ * s32), 2 = f16 (f16 x f16 -> f32).  n: 64, 128 or 256.  iters: 1 .. 65536.
+ * cycles (device, 8 bytes, 8-byte aligned, caller-owned): receives the SM
+ * clock cycles from the first issue to the completion of the last MMA (0 if
+ * the bounded wait ran out; ROTA_ERR_TIMEOUT is then recorded).  Argument
+ * errors return ROTA_ERR_INVALID_ARG synchronously. */
+rota_status rota_attn_debug_mma_cycles(int32_t kind, int32_t n, int32_t iters, uint64_t* cycles, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -257,3 +257,11 @@ def test_library_hadamard_equals_oracle(ra, n):
     else:
         assert st == ra.ROTA_OK, n
         assert np.array_equal(h, ref), n
+
+
+@pytest.mark.parametrize("kind,n,iters,ptr", [(3, 128, 8, 64), (-1, 128, 8, 64), (0, 96, 8, 64), (1, 128, 0, 64),
+                                               (2, 256, 65537, 64), (0, 64, 8, 0), (0, 64, 8, 4)])
+def test_mma_cycles_rejects_arguments_on_host(ra, kind, n, iters, ptr):
+    """Invalid kind, shape, iteration count or output pointer: refused before
+    any CUDA call (the pointers are never dereferenced)."""
+    assert ra._lib.rota_attn_debug_mma_cycles(kind, n, iters, ptr or None, None) == ra.ROTA_ERR_INVALID_ARG

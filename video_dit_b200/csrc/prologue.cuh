@@ -6,9 +6,12 @@
 // rotation inside each RoPE partition tames the partition-aligned outliers,
 // and Q, K, V are quantised to INT4 before the INT4 FlashAttention.
 //
-// One CTA per (64-token block, head, tensor in {Q, K, V}).  HBM-bound: each
-// CTA reads 64 x head_dim fp16 values once (16-byte loads) and writes
-// 64 x head_dim / 2 bytes of packed codes plus its scale(s).
+// This file holds the prologue's arithmetic (RoPE of a pair, the Walsh-Hadamard
+// units, the dense rotation of non-power-of-two blocks, the code of a value)
+// and prologue_job, the prologue of one (64-token block, head, tensor) on
+// tiles already in shared memory, which the fused QKV-projection kernel runs
+// in its epilogue.  The standalone prologue runs prologue_stream.cuh's kernel
+// when every rotation unit fits an 8-channel chunk, else prologue_kernel below.
 #pragma once
 #include <cstdint>
 #include <cuda_fp16.h>
@@ -468,6 +471,10 @@ __device__ __forceinline__ void prologue_job(const PrologueParams& p, const __ha
   }
 }
 
+// One CTA per (64-token block, head, tensor in {Q, K, V}), 5 per SM: the
+// prologue of configurations with a partition whose rotation units do not fit
+// an 8-channel chunk (they take the shared-memory rotation pass); the others
+// run prologue_stream_kernel.
 template <int D>
 __global__ void __launch_bounds__(kPrologueThreads, 5) prologue_kernel(const __grid_constant__ PrologueParams p) {
   constexpr int LD = D + 4;

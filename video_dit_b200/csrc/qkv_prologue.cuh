@@ -13,7 +13,7 @@
 // 2*H*D + h*D .. the V), fp32 accumulation, rounded to fp16 -- the fp16
 // tensors the prologue takes -- then exactly the prologue of prologue.cuh.
 //
-// One CTA = 128 tokens of one head, 256 threads.  The K loop over C: warp 0
+// One CTA = 128 tokens of one head, 256 threads; the grid is (ntiles * H, B).  The K loop over C: warp 0
 // loads the x tile (128 x 64) and the head's three W tiles (3 x D x 64) of each
 // 64-channel step with TMA (128-byte swizzle) into a 3-stage ring; warp 1
 // issues tcgen05.mma kind::f16 (Q and K as one N = 2D MMA, V as one N = D MMA,
@@ -36,6 +36,8 @@ struct QkvParams {
   PrologueParams pro; // the prologue's parameters (q, k, v unused)
   __half* v_out;      // fp16 V of the flagged heads [B,H,N,D] (NULL when none is flagged)
   int C;
+  int ntiles;         // ceil(N / 128)
+  int head_group;     // heads per raster group (see the kernel)
   uint64_t timeout_ns;
 };
 
@@ -79,7 +81,22 @@ __global__ void __launch_bounds__(kQkvThreads, 1) qkv_prologue_kernel(const __gr
   int4* sPos = reinterpret_cast<int4*>(smem + L::OFF_POS);
 
   const PrologueParams& pro = p.pro;
-  const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // Raster order: the heads are cut into groups of head_group; a group's CTAs
+  // run tile by tile with the group's heads fastest, so the CTAs resident at
+  // one time share few x tiles (each read from HBM once per group) and the
+  // group's W rows (head_group x 3 x D x C fp16) stay in L2 for the whole
+  // sweep over the tiles.
+  const int b = blockIdx.y;
+  int tile, h;
+  {
+    const int lin = blockIdx.x;
+    const int g = lin / (p.head_group * p.ntiles);
+    const int h0 = g * p.head_group;
+    const int gh = min(p.head_group, p.pro.H - h0);
+    const int r = lin - h0 * p.ntiles;
+    h = h0 + r % gh;
+    tile = r / gh;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = p.C / 64;
   const uint64_t lim = p.timeout_ns;

@@ -19,7 +19,9 @@
 #include "calib.cuh"
 #include "attn_int4.cuh"
 #include "prologue.cuh"
+#include "prologue_stream.cuh"
 #include "qkv_prologue.cuh"
+#include "mma_rate.cuh"
 
 namespace {
 
@@ -234,6 +236,35 @@ rota_status launch_int4_variant(bool g128, bool r1, dim3 grid, cudaStream_t s, c
             : launch_int4_kernel(rota::attn_int4_kernel<D, 64, false>, rota::Int4Smem<D, 64>::ALLOC, grid, s, p);
 }
 
+// The persistent prologue: as many CTAs as fit on the device at once (at most
+// one per unit), each taking a contiguous range of (batch, block, head) units.
+// The standalone prologue.  When every partition's rotation units fit an
+// 8-channel chunk: the persistent kernel, as many CTAs as fit on the device
+// at once (at most one per unit), each taking a contiguous range of (batch,
+// block, head) units.  Otherwise the kernel with one CTA per (block, head,
+// tensor), whose shared-memory rotation pass those partitions need.
+template <int D>
+rota_status launch_prologue(int units, cudaStream_t s, const rota::PrologueParams& p) {
+  if (p.any_unfused) {
+    const dim3 grid(p.nblk, p.H, units / (p.H * p.nblk) * 3);
+    rota::prologue_kernel<D><<<grid, rota::kPrologueThreads, 0, s>>>(p);
+    return cuda_status(cudaGetLastError());
+  }
+  using L = rota::StreamSmem<D>;
+  auto kernel = rota::prologue_stream_kernel<D>;
+  rota_status st = set_smem(kernel, L::BYTES);
+  if (st != ROTA_OK) return st;
+  int dev = 0, nsm = 0, per_sm = 0;
+  if ((st = cuda_status(cudaGetDevice(&dev))) != ROTA_OK) return st;
+  if ((st = cuda_status(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev))) != ROTA_OK) return st;
+  if ((st = cuda_status(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, rota::kPrologueThreads,
+                                                                     L::BYTES))) != ROTA_OK)
+    return st;
+  const int grid = std::max(1, std::min(units, nsm * std::max(per_sm, 1)));
+  kernel<<<grid, rota::kPrologueThreads, L::BYTES, s>>>(p, units, kDefaultTimeoutNs);
+  return cuda_status(cudaGetLastError());
+}
+
 }  // namespace
 
 namespace {
@@ -389,16 +420,11 @@ rota_status rota_attn_prepare_qk(const rota_attn_desc* d, const uint16_t* q, con
   p.q = reinterpret_cast<const __half*>(q);
   p.k = reinterpret_cast<const __half*>(k);
   p.v = reinterpret_cast<const __half*>(v);
-  const dim3 grid(p.nblk, d->H, d->B * 3);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d->head_dim == 128)
-    rota::prologue_kernel<128><<<grid, rota::kPrologueThreads, 0, s>>>(p);
-  else
-    rota::prologue_kernel<64><<<grid, rota::kPrologueThreads, 0, s>>>(p);
-  return cuda_status(cudaGetLastError());
+  const int units = d->B * d->H * p.nblk;
+  return d->head_dim == 128 ? launch_prologue<128>(units, s, p) : launch_prologue<64>(units, s, p);
 }
 
-// part: 1 = widen only, 2 = attention only, 3 = both
 rota_status rota_attn_qkv_prepare(const rota_attn_desc* d, const uint16_t* x, const uint16_t* w, int32_t C,
                                   const uint8_t* head_flags, const rota_attn_buffers* buf, uint16_t* v_out,
                                   void* stream) {
@@ -426,7 +452,12 @@ rota_status rota_attn_qkv_prepare(const rota_attn_desc* d, const uint16_t* x, co
   if ((st = make_fp16_map(&p.tm_x, x, static_cast<uint64_t>(d->B) * d->N, C, 128)) != ROTA_OK) return st;
   if ((st = make_fp16_map(&p.tm_w, w, static_cast<uint64_t>(3) * d->H * D, C, static_cast<uint32_t>(D))) != ROTA_OK)
     return st;
-  const dim3 grid((d->N + 127) / 128, d->H, d->B);
+  // heads per raster group: the group's W rows should take at most ~40 MB of L2
+  const long long w_head = 3ll * D * C * 2;
+  const int ngroups = static_cast<int>((d->H * w_head + (40ll << 20) - 1) / (40ll << 20));
+  p.ntiles = (d->N + 127) / 128;
+  p.head_group = (d->H + ngroups - 1) / ngroups;
+  const dim3 grid(p.ntiles * d->H, d->B);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (D == 128) {
     if ((st = set_smem(rota::qkv_prologue_kernel<128>, rota::QkvSmem<128>::ALLOC)) != ROTA_OK) return st;
@@ -438,6 +469,7 @@ rota_status rota_attn_qkv_prepare(const rota_attn_desc* d, const uint16_t* x, co
   return cuda_status(cudaGetLastError());
 }
 
+// part: 1 = widen only, 2 = attention only, 3 = both
 static rota_status launch_int4(const rota_attn_desc* d, const rota_attn_buffers* buf, const uint8_t* head_flags,
                                float* out, void* stream, bool dump, int b, int h, int r0, int nr, int32_t* s_out,
                                uint8_t* p_out, int part = 3) {
@@ -812,6 +844,17 @@ rota_status rota_attn_debug_hadamard(int32_t n, int8_t* h) {
   for (int i = 0; i < n; ++i)
     for (int j = 0; j < n; ++j) h[i * n + j] = ((neg[i] >> j) & 1ull) ? -1 : 1;
   return ROTA_OK;
+}
+
+rota_status rota_attn_debug_mma_cycles(int32_t kind, int32_t n, int32_t iters, uint64_t* cycles, void* stream) {
+  if (kind < 0 || kind > 2 || (n != 64 && n != 128 && n != 256) || iters < 1 || iters > 65536 || !cycles ||
+      reinterpret_cast<uintptr_t>(cycles) % 8 != 0)
+    return ROTA_ERR_INVALID_ARG;
+  rota_status st = set_smem(rota::mma_rate_kernel, rota::kRateSmem);
+  if (st != ROTA_OK) return st;
+  rota::mma_rate_kernel<<<1, rota::kRateThreads, rota::kRateSmem, static_cast<cudaStream_t>(stream)>>>(
+      kind, n, iters, kDefaultTimeoutNs, reinterpret_cast<unsigned long long*>(cycles));
+  return cuda_status(cudaGetLastError());
 }
 
 rota_status rota_attn_debug_inject_timeout(int32_t arm, uint64_t timeout_ns) {

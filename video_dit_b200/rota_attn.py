@@ -65,6 +65,7 @@ _SIGS = {
                                    ctypes.c_int32, _P, _P, _P, _P], ctypes.c_int),
     "rota_attn_debug_pcode": ([_P, _P, ctypes.c_int64, _P], ctypes.c_int),
     "rota_attn_debug_inject_timeout": ([ctypes.c_int32, ctypes.c_uint64], ctypes.c_int),
+    "rota_attn_debug_mma_cycles": ([ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P], ctypes.c_int),
     "rota_attn_fwd_int4_noalloc": ([_D, _P, _P, _P, _P, _P], ctypes.c_int),
     "rota_attn_pipeline_create": ([ctypes.c_int32, ctypes.POINTER(_P)], ctypes.c_int),
     "rota_attn_pipeline_destroy": ([_P], ctypes.c_int),
@@ -230,6 +231,10 @@ def rota_attn_debug_hadamard(n: int):
     """-> (status, int8 [n, n]): the library's Hadamard matrix of a non-power-of-two order."""
     h = np.zeros((max(n, 1), max(n, 1)), np.int8)
     return _lib.rota_attn_debug_hadamard(int(n), h.ctypes.data), h
+
+
+def rota_attn_debug_mma_cycles(kind: int, n: int, iters: int, cycles, stream=None) -> int:
+    return _lib.rota_attn_debug_mma_cycles(int(kind), int(n), int(iters), _ptr(cycles), _stream(stream))
 
 
 def rota_attn_debug_inject_timeout(arm: bool, timeout_ns: int = 0) -> int:
