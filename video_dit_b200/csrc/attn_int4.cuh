@@ -111,8 +111,8 @@ struct Int4Smem {
   static constexpr int SPILL_BYTES = G == 128 ? 2 * kBM * kBN * 4 : 0;
   static constexpr int OFF_BAR = OFF_SPILL + SPILL_BYTES;
   // barriers: op_full[OPS] op_empty[OPS] q_full s_full[2] s_empty[2]
-  //           p_full[2][2] p_empty[2][2] acc_full acc_empty l_full mma_done[2] turn[2]
-  static constexpr int NBAR = 2 * OPS + 1 + 2 + 2 + 4 + 4 + 1 + 1 + 1 + 2 + 2;
+  //           p_full[2][2] p_empty[2][2] acc_full acc_empty l_full mma_done[2]
+  static constexpr int NBAR = 2 * OPS + 1 + 2 + 2 + 4 + 4 + 1 + 1 + 1 + 2;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int BYTES = OFF_ABORT + 4;
@@ -286,9 +286,6 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
   uint64_t* acc_empty = acc_full + 1;           // 4 correction warps hold ACC in registers
   uint64_t* l_full = acc_empty + 1;             // 8 softmax warps wrote their rows' l
   uint64_t* mma_done = l_full + 1;              // [2], one per issuing warp
-  // turn[t]: the other tile's 4 softmax warps finished a code phase, so tile
-  // t may take the exponential unit for its next one
-  uint64_t* turn = mma_done + 2;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + L::OFF_ABORT);
   float* sTau = reinterpret_cast<float*>(smem + L::OFF_TAU);
@@ -324,8 +321,6 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     mbar_init(l_full, 8);
     mbar_init(&mma_done[0], 1);
     mbar_init(&mma_done[1], 1);
-    mbar_init(&turn[0], 4);
-    mbar_init(&turn[1], 4);
     *sAbort = 0;
     fence_mbar_init();
   }
@@ -536,21 +531,6 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     // the key scales are read one block (pair) ahead
     float sk_next = __ldg(ksc), sk_next2 = nkb > 1 ? __ldg(ksc + 1) : 0.f;
 
-    // The two tiles take turns on the code phase (the exponentials): while
-    // one tile's warps code a block, the other tile's warps load, reduce and
-    // store theirs, so the exponential unit is not split between two phases
-    // in lockstep.  Tile 0 goes first.
-    int turns = 0;
-    auto my_turn = [&]() -> bool {
-      const bool ok = warp_wait(&turn[t], turns & 1, lim);
-      ++turns;
-      return ok;
-    };
-    auto pass_turn = [&]() {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&turn[t ^ 1]);
-    };
-    if (t == 1) pass_turn();
 
     float m = -INFINITY, l = 0.f;
     bool aborted = false;
@@ -565,10 +545,8 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         const float m_old = m;
         m = fmaxf(m, __fmul_rn(smax, c18));
         uint32_t pw[kBN / 4];
-        if (!my_turn()) { aborted = true; break; }
         const float lsum = nvalid == kBN ? block_codes_l<false, R1>(sr, nvalid, c18, m, pw, sTau)
                                          : block_codes_l<true, R1>(sr, nvalid, c18, m, pw, sTau);
-        pass_turn();
         const float alpha = alpha_of(j == 0, m_old, m);
         l = __fmaf_rn(l, alpha, lsum);
         if (!emit(j, pw, alpha)) { aborted = true; break; }
@@ -605,7 +583,6 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         const float alpha = alpha_of(j0 == 0, m_old, m);
         uint32_t pw[kBN / 4];
         float lsum1 = 0.f;
-        if (!my_turn()) { aborted = true; break; }
         if (has1) {
           lsum1 = nv1 == kBN ? block_codes_l<false, R1>(sr, nv1, c1, m, pw, sTau)
                              : block_codes_l<true, R1>(sr, nv1, c1, m, pw, sTau);
@@ -621,7 +598,6 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         }
         const float lsum0 = nv0 == kBN ? block_codes_l<false, R1>(sr, nv0, c0, m, pw, sTau)
                                        : block_codes_l<true, R1>(sr, nv0, c0, m, pw, sTau);
-        pass_turn();
         l = __fadd_rn(__fmaf_rn(l, alpha, lsum0), lsum1);
         if (!emit(j0, pw, alpha)) { aborted = true; break; }
         if (warp_flag(sAbort)) { aborted = true; break; }
@@ -649,19 +625,28 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         if (!warp_wait(acc_full, u & 1, lim)) { aborted = true; break; }
         tc_fence_after();
         const uint32_t tO = tmem + L::T_O + t * kBM + t_lane;
-        // the block's ACC, all 128 query columns
+        // the block's ACC, all 128 query columns, and the first half of O
         uint32_t a[kBM];
+        uint32_t oh[64];
         {
           uint32_t(&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&a[0]);
           uint32_t(&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&a[32]);
           uint32_t(&a2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&a[64]);
           uint32_t(&a3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&a[96]);
+          uint32_t(&q0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&oh[0]);
+          uint32_t(&q1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&oh[32]);
+          tmem_st_wait();   // this thread's O stores of the previous tile-block are complete
           tmem_ld32(tA, a0);
           tmem_ld32(tA + 32, a1);
           tmem_ld32(tA + 64, a2);
           tmem_ld32(tA + 96, a3);
+          if (j > 0) {
+            tmem_ld32(tO, q0);
+            tmem_ld32(tO + 32, q1);
+          }
           tmem_wait_dep2(a0, a1);
           tmem_wait_dep2(a2, a3);
+          tmem_wait_dep2(q0, q1);
         }
         // ACC is in registers: the next P V may overwrite it
         tc_fence_before();
@@ -673,17 +658,8 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         const int* fl = sFlag + (2 * t + sl) * 4;
         const bool moved = j > 0 && (fl[0] | fl[1] | fl[2] | fl[3]) != 0;
         const float* al = sAlpha + (2 * t + sl) * kBM;
-        // O in two 64-column halves: one load round trip and two stores each
-#pragma unroll
-        for (int hb = 0; hb < kBM / 64; ++hb) {
-          uint32_t o[64];
-          uint32_t(&o0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
-          uint32_t(&o1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[32]);
-          if (j > 0) {
-            tmem_ld32(tO + 64 * hb, o0);
-            tmem_ld32(tO + 64 * hb + 32, o1);
-            tmem_wait_dep2(o0, o1);
-          }
+        // O in two 64-column halves (the first already loaded): FMAs, then two stores
+        auto half = [&](int hb, uint32_t(&o)[64]) {
           if (j == 0) {
 #pragma unroll
             for (int i = 0; i < 64; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(a[64 * hb + i]), s18));
@@ -712,16 +688,29 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
               o[i + 1] = __float_as_uint(x1);
             }
           }
-          tmem_st32(tO + 64 * hb, o0);
-          tmem_st32(tO + 64 * hb + 32, o1);
+          tmem_st32(tO + 64 * hb, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+          tmem_st32(tO + 64 * hb + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+        };
+        half(0, oh);
+        {
+          uint32_t o[64];
+          uint32_t(&o0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
+          uint32_t(&o1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[32]);
+          if (j > 0) {
+            tmem_ld32(tO + 64, o0);
+            tmem_ld32(tO + 96, o1);
+            tmem_wait_dep2(o0, o1);
+          }
+          half(1, o);
         }
-        tmem_st_wait();
-        // this tile's codes and alpha of block j are consumed
+        // this tile's codes and alpha of block j are consumed (the O stores
+        // may still be in flight: they are waited for before O is read again)
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_empty[2 * t + sl]);
       }
       if (warp_flag(sAbort)) aborted = true;
     }
+    tmem_st_wait();
     // ---- epilogue: out = O / l once every row's l is final ----
     if (!aborted && !warp_wait(l_full, 0, lim)) aborted = true;
     if (aborted || warp_flag(sAbort)) {
