@@ -132,11 +132,12 @@ def workload_config(w, l2_note):
 # ----------------------------------------------------------- CPU oracle ---
 
 # DRAM bytes (read + write) per attention launch, from one ncu capture of the
-# current kernels on the F = 3 sweep point (B=1, H=40, N=4680, profiles/), per
-# (head, token): the traffic is the K/V images or tiles and the output, linear
-# in B * heads * N.  A kernel missing here has no capture of its current
-# version, and its traffic is reported as null.
-TRAFFIC_PER_HEAD_TOKEN = {"attn_int4_kernel": 586.5, "attn_fp16_kernel": 1076.75}
+# current kernels per (head, token): the INT4 kernel on the F = 11 sweep point
+# (B=1, H=40, N=17160, whose output and operand images exceed L2), the FP16
+# kernel on the F = 3 point (profiles/).  The traffic is the K/V images or
+# tiles and the output, linear in B * heads * N.  A kernel missing here has no
+# capture of its current version, and its traffic is reported as null.
+TRAFFIC_PER_HEAD_TOKEN = {"attn_int4_kernel": 772.9, "attn_fp16_kernel": 1076.75}
 
 
 def traffic_per_launch(kernel, w, heads):

@@ -354,10 +354,9 @@ const char* rota_attn_status_string(rota_status s);
  * ROTA_NOALLOC_MAX_TABLE floats; larger problems return
  * ROTA_ERR_UNSUPPORTED, with nothing enqueued.
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current and keeps it; make that
- * first call before any stream capture.  A device reset (cudaDeviceReset)
- * invalidates the kept address: after one, do not call this entry point
- * again in the same process.  The RoPE tables are copied from a static host
+ * (cudaGetSymbolAddress) with that device current and keeps it.  A device
+ * reset (cudaDeviceReset) invalidates the kept address: after one, do not
+ * call this entry point again in the same process.  The RoPE tables are copied from a static host
  * buffer with a pageable cudaMemcpyAsync, which synchronises `stream` first.
  * All calls share the one array and it keeps the last call's contents (every
  * byte a call reads is written earlier in the same call, so nothing has to

@@ -193,3 +193,31 @@ def test_pcode_function_exhaustive_range():
         bad = (u[:n] != want).nonzero()
         assert bad.numel() == 0, (b0, d[bad[:5, 0]].cpu().numpy(), u[bad[:5, 0]].cpu().numpy(),
                                   want[bad[:5, 0]].cpu().numpy())
+
+
+def test_prologue_multi_unit_ranges_batch_and_flags():
+    """B = 2, H = 8, N = 1560 (25 blocks): 400 (batch, block, head) units, more
+    than the prologue's persistent CTAs, so CTAs take ranges of one or two
+    units that cross heads, blocks and the batch boundary; heads 3 and 6 are
+    flagged (their Q / K come out RoPE'd in fp16, their V job is skipped).
+    Codes and scales of the INT4 heads and the RoPE'd rows of the flagged
+    heads byte-exact against the oracle."""
+    from gpu_util import desc_of, lib, to_dev
+    w = synth.scaled(synth.WORKLOADS["wan480"], "multi_unit", B=2, H=8, grid=(4, 15, 26))
+    q, k, v = synth.make_inputs(w)
+    flags = np.zeros(w.H, np.uint8)
+    flags[[3, 6]] = 1
+    ra = lib()
+    att = ra.RotaAttention(desc_of(w), need_fp16=True)
+    att.prepare(to_dev(q), to_dev(k), to_dev(v), flags)
+    assert ra.rota_attn_get_error() == ra.ROTA_OK
+    codes = {k_: (None if t is None else t.cpu().numpy()) for k_, t in att.codes().items()}
+    ref = _oracle(w, q, k, v, flags)
+    int4 = [h for h in range(w.H) if not flags[h]]
+    for key in ("q_codes", "k_codes", "v_codes"):
+        assert np.array_equal(codes[key][:, int4], ref[key][:, int4]), key
+    for key in ("q_scale", "k_scale", "v_scale"):
+        assert np.array_equal(codes[key][:, int4].view(np.uint32), ref[key][:, int4].view(np.uint32)), key
+    for h in (3, 6):
+        assert np.array_equal(codes["q_rope"].view(np.uint16)[:, h], ref["q_rope"][:, h]), h
+        assert np.array_equal(codes["k_rope"].view(np.uint16)[:, h], ref["k_rope"][:, h]), h

@@ -121,6 +121,7 @@ def test_rope_rounding_order_bit_exact(rope_dim, grid):
     toks = [0, 1, W, Hh * W, T * Hh * W - 1] + list(rng.integers(0, T * Hh * W, 40))
     halves = [r // 2 for r in rope_dim]
     toff = [0, T * halves[0], T * halves[0] + Hh * halves[1]]
+    fused_differs = 0
     for n in toks:
         n = int(n)
         pos = (n // (Hh * W), (n // W) % Hh, n % W)
@@ -135,8 +136,14 @@ def test_rope_rounding_order_bit_exact(rope_dim, grid):
                 x0, x1 = np.float32(x[off + 2 * i]), np.float32(x[off + 2 * i + 1])
                 want[off + 2 * i] = np.float32(np.float32(x0 * c) - np.float32(x1 * s_))
                 want[off + 2 * i + 1] = np.float32(np.float32(x0 * s_) + np.float32(x1 * c))
+                # the contracted form fma(x0, c, -RN(x1 s)): the fp32 product is
+                # exact in double, so one rounding of the double difference
+                fz = np.float32(np.float64(x0) * np.float64(c) - np.float64(np.float32(x1 * s_)))
+                fused_differs += int(fz != want[off + 2 * i])
             off += rope_dim[a]
         assert np.array_equal(got.view(np.uint32), want.view(np.uint32)), n
+    # the check can tell: a contracted multiply-add gives other bits on these rows
+    assert fused_differs > 0
 
 
 def test_unquantised_reference_matches_torch_sdpa_float64():
@@ -512,6 +519,22 @@ def test_single_group_is_global_max():
     deq = (vc * p["v_scale"][0, 0].astype(np.float64)[:, :, None]).transpose(0, 2, 1).reshape(-1, w.d)
     want = (u.astype(np.float64) @ deq[: w.N]) / u.sum(axis=1, keepdims=True)
     assert np.abs(out - want).max() < 1e-12
+
+
+def test_max_group_128_is_global_max_below_129_keys():
+    """With N <= 128 keys a 128-key group holds every key, so the codes and the
+    output equal those of the single global group, bit for bit."""
+    w = synth.scaled(synth.WORKLOADS["wan480"], "g128", H=1, grid=(1, 2, 50))   # N = 100
+    q, k, v = synth.make_inputs(w)
+    p = oracle.prepare(q, k, v, w.grid, w.rope_dim, w.had_block)
+    sm = 1 / math.sqrt(w.d)
+    o128, s128, u128 = oracle.attn_int4(p, w.N, sm, 0, 0, 0, w.N, group=128, dump=True)
+    og, sg, ug = oracle.attn_int4(p, w.N, sm, 0, 0, 0, w.N, group=1 << 20, dump=True)
+    assert np.array_equal(u128, ug) and np.array_equal(s128, sg)
+    assert np.array_equal(o128, og)
+    # and the 64-key reading differs on these rows (the pin can tell them apart)
+    _, _, u64 = oracle.attn_int4(p, w.N, sm, 0, 0, 0, w.N, group=64, dump=True)
+    assert not np.array_equal(u64, ug)
 
 
 def test_fp16_path_matches_torch_sdpa_float64():

@@ -629,24 +629,16 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         uint32_t a[kBM];
         uint32_t oh[64];
         {
-          uint32_t(&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&a[0]);
-          uint32_t(&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&a[32]);
-          uint32_t(&a2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&a[64]);
-          uint32_t(&a3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&a[96]);
-          uint32_t(&q0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&oh[0]);
-          uint32_t(&q1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&oh[32]);
+          uint32_t(&aa)[64] = *reinterpret_cast<uint32_t(*)[64]>(&a[0]);
+          uint32_t(&ab)[64] = *reinterpret_cast<uint32_t(*)[64]>(&a[64]);
           tmem_st_wait();   // this thread's O stores of the previous tile-block are complete
-          tmem_ld32(tA, a0);
-          tmem_ld32(tA + 32, a1);
-          tmem_ld32(tA + 64, a2);
-          tmem_ld32(tA + 96, a3);
-          if (j > 0) {
-            tmem_ld32(tO, q0);
-            tmem_ld32(tO + 32, q1);
-          }
-          tmem_wait_dep2(a0, a1);
-          tmem_wait_dep2(a2, a3);
-          tmem_wait_dep2(q0, q1);
+          tmem_ld64(tA, aa);   // 64-column loads and stores: fewer, larger TMEM accesses
+          tmem_ld64(tA + 64, ab);
+          if (j > 0) tmem_ld64(tO, oh);
+          tmem_ld_wait();
+          tmem_dep64(aa);
+          tmem_dep64(ab);
+          tmem_dep64(oh);
         }
         // ACC is in registers: the next P V may overwrite it
         tc_fence_before();
@@ -688,18 +680,15 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
               o[i + 1] = __float_as_uint(x1);
             }
           }
-          tmem_st32(tO + 64 * hb, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
-          tmem_st32(tO + 64 * hb + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+          tmem_st64(tO + 64 * hb, o);
         };
         half(0, oh);
         {
           uint32_t o[64];
-          uint32_t(&o0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
-          uint32_t(&o1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[32]);
           if (j > 0) {
-            tmem_ld32(tO + 64, o0);
-            tmem_ld32(tO + 96, o1);
-            tmem_wait_dep2(o0, o1);
+            tmem_ld64(tO + 64, o);
+            tmem_ld_wait();
+            tmem_dep64(o);
           }
           half(1, o);
         }
