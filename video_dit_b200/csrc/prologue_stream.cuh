@@ -32,17 +32,18 @@
 
 namespace rota {
 
-template <int D>
+template <int D, int NT>
 struct StreamSmem {
+  static constexpr int NW = NT / 32;                // warps
   static constexpr int TILE = 64 * D * 2;           // one fp16 tile
   static constexpr int NS = D == 128 ? 4 : 6;       // ring stages
-  static constexpr int RG = D == 128 ? 4 : 8;       // V row groups
+  static constexpr int RG = NW / (D / 64);          // V row groups (D / 64 warps each)
   static constexpr int OFF_TILE = 0;
   static constexpr int OFF_ANG = NS * TILE;         // float2 [64 tokens][D/2 pairs]: (cos, sin)
   static constexpr int OFF_VST = OFF_ANG + 64 * (D / 2) * 8;   // V codes [D channels][32 bytes], swizzled slots
   static constexpr int OFF_VRED = OFF_VST + D * 32;  // float [RG][D]: per row group channel max
-  static constexpr int OFF_RED = OFF_VRED + RG * D * 4;         // float [2][2][8]: Q/K warp max, two parities
-  static constexpr int OFF_POS = OFF_RED + 2 * 2 * 8 * 4;       // int4 [64]: token coordinates
+  static constexpr int OFF_RED = OFF_VRED + RG * D * 4;         // float [2][2][NW]: Q/K warp max, two parities
+  static constexpr int OFF_POS = OFF_RED + 2 * 2 * NW * 4;      // int4 [64]: token coordinates
   static constexpr int OFF_BAR = OFF_POS + 64 * 16;             // uint64 [NS]
   static constexpr int BYTES = OFF_BAR + NS * 8;
   static_assert(2 * (BYTES + 1024) <= 233472, "two CTAs per SM");
@@ -135,18 +136,19 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kPrologueThreads, 2)
+template <int D, int NT>
+__global__ void __launch_bounds__(NT, 2)
     prologue_stream_kernel(const __grid_constant__ PrologueParams p, int units, uint64_t timeout_ns) {
-  using L = StreamSmem<D>;
+  using L = StreamSmem<D, NT>;
+  constexpr int NW = L::NW;
   constexpr int NS = L::NS;
   constexpr int CH = D / 8;                        // 8-channel chunks per row
-  constexpr int RSTEP = kPrologueThreads / CH;     // rows between a thread's rows
+  constexpr int RSTEP = NT / CH;     // rows between a thread's rows
   constexpr int PER = 64 / RSTEP;                  // rows per thread
   constexpr int WPR = D / 64;                      // V: warps per row group (32 channel pairs each)
   constexpr int RG = L::RG, RPG = 64 / RG;         // V: row groups, rows per group
-  static_assert(CH * RSTEP == kPrologueThreads && PER * RSTEP == 64, "Q/K split");
-  static_assert(WPR * RG == kPrologueThreads / 32 && RPG % 8 == 0, "V split");
+  static_assert(CH * RSTEP == NT && PER * RSTEP == 64, "Q/K split");
+  static_assert(WPR * RG == NT / 32 && RPG % 8 == 0, "V split");
 
   extern __shared__ __align__(128) uint8_t sm[];
   uint8_t* tiles = sm + L::OFF_TILE;
@@ -218,7 +220,7 @@ __global__ void __launch_bounds__(kPrologueThreads, 2)
       }
       __syncthreads();
 #pragma unroll 4
-      for (int e = tid; e < 64 * (D / 2); e += kPrologueThreads) {
+      for (int e = tid; e < 64 * (D / 2); e += NT) {
         const int r = e / (D / 2), c = 2 * (e % (D / 2));
         const int a = c < p.coff[1] ? 0 : (c < p.coff[2] ? 1 : 2);
         const int4 ps = sPos[r];
@@ -289,11 +291,11 @@ __global__ void __launch_bounds__(kPrologueThreads, 2)
         }
       mq = warp_max(mq);
       mk = warp_max(mk);
-      float* rd = red + (nred & 1) * 16;
+      float* rd = red + (nred & 1) * 2 * NW;
       ++nred;
       if (lane == 0) {
         rd[warp] = mq;
-        rd[8 + warp] = mk;
+        rd[NW + warp] = mk;
       }
       if (!__syncthreads_and(ok)) return;   // also: the Q and K stages are read
       if (tid == 0) {
@@ -301,9 +303,9 @@ __global__ void __launch_bounds__(kPrologueThreads, 2)
         issue();
       }
 #pragma unroll
-      for (int w = 0; w < 8; ++w) {
+      for (int w = 0; w < NW; ++w) {
         mq = fmaxf(mq, rd[w]);
-        mk = fmaxf(mk, rd[8 + w]);
+        mk = fmaxf(mk, rd[NW + w]);
       }
       const float iq = mq == 0.f ? 0.f : __fdiv_rn(7.f, mq);
       const float ik = mk == 0.f ? 0.f : __fdiv_rn(7.f, mk);
@@ -379,7 +381,7 @@ __global__ void __launch_bounds__(kPrologueThreads, 2)
       // 16-byte pieces of the block's D x 32 code bytes, in memory order
       uint8_t* vdst = p.v_codes + (head * p.nblk + blk) * D * 32;
 #pragma unroll
-      for (int t = tid; t < D * 2; t += kPrologueThreads) {
+      for (int t = tid; t < D * 2; t += NT) {
         const int c = t >> 1, hh = t & 1;
         const int sw = (c >> 1) & (RG - 1);
         const uint8_t* src = vst + c * 32;
