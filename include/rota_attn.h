@@ -394,6 +394,12 @@ rota_status rota_attn_debug_dump_int4(const rota_attn_desc* desc, const rota_att
  * device uint8), so it can be checked exhaustively against the definition. */
 rota_status rota_attn_debug_pcode(const float* d, uint8_t* u, int64_t n, void* stream);
 
+/* The same P-code function with the exponential taken on the FMA pipe
+ * (Cody-Waite split and a fitted polynomial, the path the INT4 kernel can
+ * route a share of the keys through) instead of the exponential unit; same
+ * arguments, errors and result (the exact code) as rota_attn_debug_pcode. */
+rota_status rota_attn_debug_pcode_fma(const float* d, uint8_t* u, int64_t n, void* stream);
+
 /* Fault injection for the bounded waits: the next INT4 launch skips its first
  * score MMA, so every wait on it runs out after `timeout_ns` and the kernel
  * exits with ROTA_ERR_TIMEOUT.  One-shot; 0 disarms. */

@@ -88,6 +88,7 @@ def test_null_arguments_rejected_on_host(ra):
     assert ra._lib.rota_attn_fwd_int4(ctypes.byref(d), ctypes.byref(b), None, None, None) == 1
     assert ra._lib.rota_attn_fwd_fp16_fallback(ctypes.byref(d), ctypes.byref(b), None, None, None, None) == 1
     assert ra._lib.rota_attn_debug_pcode(None, None, 5, None) == 1
+    assert ra._lib.rota_attn_debug_pcode_fma(None, None, 5, None) == 1
     assert ra._lib.rota_attn_prepare_qk(None, None, None, None, None, None, None) == 1
     assert ra.rota_attn_status_string(4) == "device wait timed out"
 

@@ -110,7 +110,11 @@ def test_fp16_fallback_heads(name):
         assert row_stats(out[0, h], o_ref)[0] <= TOL
 
 
-def test_pcode_function_matches_oracle_dense():
+PCODE_ENTRIES = ["rota_attn_debug_pcode", "rota_attn_debug_pcode_fma"]   # exponential on MUFU / on the FMA pipe
+
+
+@pytest.mark.parametrize("entry", PCODE_ENTRIES)
+def test_pcode_function_matches_oracle_dense(entry):
     import torch
     from gpu_util import lib
     ra = lib()
@@ -119,11 +123,12 @@ def test_pcode_function_matches_oracle_dense():
                         np.float32([-1.0, 0.0, -0.0, -5.0, -4.906890, -30.0, 1e-7])])
     dd = torch.from_numpy(d).cuda()
     u = torch.empty(d.size, dtype=torch.uint8, device="cuda")
-    ra._check(ra.rota_attn_debug_pcode(dd, u), "pcode")
+    ra._check(getattr(ra, entry)(dd, u), "pcode")
     assert np.array_equal(u.cpu().numpy(), oracle.pcode_array(d))
 
 
-def test_pcode_function_exhaustive_near_thresholds():
+@pytest.mark.parametrize("entry", PCODE_ENTRIES)
+def test_pcode_function_exhaustive_near_thresholds(entry):
     """Every fp32 within 2^16 ulps of each of the 15 code thresholds: the
     band in which the kernel re-decides a code exactly must cover every
     estimate that could round the wrong way."""
@@ -140,7 +145,7 @@ def test_pcode_function_exhaustive_near_thresholds():
     d = d[d <= 0]
     dd = torch.from_numpy(d).cuda()
     u = torch.empty(d.size, dtype=torch.uint8, device="cuda")
-    ra._check(ra.rota_attn_debug_pcode(dd, u), "pcode")
+    ra._check(getattr(ra, entry)(dd, u), "pcode")
     assert np.array_equal(u.cpu().numpy(), oracle.pcode_array(d))
 
 
@@ -160,7 +165,8 @@ def test_int4_long_sequence_sampled_rows():
     assert row_stats(out[0, 0, :64], o0)[0] <= TOL
 
 
-def test_pcode_function_exhaustive_range():
+@pytest.mark.parametrize("entry", PCODE_ENTRIES)
+def test_pcode_function_exhaustive_range(entry):
     """Every fp32 d in [-6, -0] (about 1.1e9 values): the kernel's P-code
     function against the oracle's, via the oracle's own decision boundaries
     (u(d) is a step function of d, so 15 boundary values pin it everywhere)."""
@@ -188,7 +194,7 @@ def test_pcode_function_exhaustive_range():
         n = min(chunk, hi + 1 - b0)
         bits = torch.arange(b0 - (1 << 32), b0 - (1 << 32) + n, dtype=torch.int32, device="cuda")
         d = bits.view(torch.float32)
-        ra._check(ra.rota_attn_debug_pcode(d, u[:n]), "pcode")
+        ra._check(getattr(ra, entry)(d, u[:n]), "pcode")
         want = torch.bucketize(d, tau, right=True).to(torch.uint8)
         bad = (u[:n] != want).nonzero()
         assert bad.numel() == 0, (b0, d[bad[:5, 0]].cpu().numpy(), u[bad[:5, 0]].cpu().numpy(),

@@ -152,6 +152,55 @@ __device__ __forceinline__ uint32_t pcode(float d, const float* tau) {
   return u < 15u ? u : 15u;
 }
 
+// 2^d on the FMA pipe (d <= 0), for a share of the keys: a Cody-Waite split
+// d = n + f with n = rne(d) (the 1.5 * 2^23 addition; f = d - n in [-1/2, 1/2]
+// exactly) and a degree-6 polynomial for 2^f whose coefficients were fitted
+// for this kernel to the relative error of 2^f on [-1/2, 1/2] (weighted least
+// squares at Chebyshev nodes, reweighted toward equal ripple, rounded to
+// fp32): with one rounding per Horner step its relative error is below
+// 8.5e-8 (2^-23.5), inside the 2^-22 the code decision assumes of
+// ex2.approx, so the same two-rounding test and the same exact fallback
+// apply.  2^n enters through the exponent field; d is clamped at -100 (the
+// code is 0 there and 2^-100 is still a normal number).
+constexpr float kP0 = 1.0f, kP1 = 0.6931471824645996f, kP2 = 0.24022646248340607f, kP3 = 0.05550328642129898f,
+                kP4 = 0.009618489071726799f, kP5 = 0.0013399930903688073f, kP6 = 0.0001534580806037411f;
+__device__ __forceinline__ void ex2_fma2(float d0, float d1, float& e0, float& e1) {
+  d0 = fmaxf(d0, -100.f);
+  d1 = fmaxf(d1, -100.f);
+  float t0, t1, n0, n1, f0, f1;
+  add2(t0, t1, d0, d1, 12582912.f, 12582912.f);      // 1.5 * 2^23 + rne(d)
+  add2(n0, n1, t0, t1, -12582912.f, -12582912.f);    // rne(d), exact
+  add2(f0, f1, d0, d1, -n0, -n1);                    // d - n, exact
+  float p0 = kP6, p1 = kP6;
+  fma2(p0, p1, p0, p1, f0, f1, kP5, kP5);
+  fma2(p0, p1, p0, p1, f0, f1, kP4, kP4);
+  fma2(p0, p1, p0, p1, f0, f1, kP3, kP3);
+  fma2(p0, p1, p0, p1, f0, f1, kP2, kP2);
+  fma2(p0, p1, p0, p1, f0, f1, kP1, kP1);
+  fma2(p0, p1, p0, p1, f0, f1, kP0, kP0);
+  e0 = __int_as_float(__float_as_int(p0) + ((__float_as_int(t0) - 0x4B400000) << 23));
+  e1 = __int_as_float(__float_as_int(p1) + ((__float_as_int(t1) - 0x4B400000) << 23));
+}
+
+// The P code of d with the exponential taken on the FMA pipe (the function
+// the main loop applies to the keys routed there; pcode() above for the rest).
+__device__ __forceinline__ uint32_t pcode_fma(float d, const float* tau) {
+  float e, e_unused;
+  ex2_fma2(d, d, e, e_unused);
+  const uint32_t lo = __float_as_uint(__fmaf_rn(e, kLo, kMag)) - kMagBits;
+  const uint32_t hi = __float_as_uint(__fmaf_rn(e, kHi, kMag)) - kMagBits;
+  uint32_t u = lo;
+  if (lo != hi && hi <= 15u && d >= tau[hi]) u = hi;
+  return u < 15u ? u : 15u;
+}
+
+// Of every four 4-key groups of a block, the first kExpFmaGroups take their
+// exponentials on the FMA pipe, the rest on MUFU (measured: a share of the
+// exponentials moved to the FMA pipe does not shorten this kernel, whose
+// exponential unit is a quarter busy -- see the design notes; 0 keeps all on
+// MUFU).
+constexpr int kExpFmaGroups = 0;
+
 __device__ __forceinline__ void setmaxnreg_issue() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 32;" ::: "memory");
 }
@@ -223,7 +272,16 @@ __device__ __forceinline__ uint32_t block_codes(const uint32_t (&sr)[kBN], int n
       if (k + 2 >= nvalid) d2 = -INFINITY;
       if (k + 3 >= nvalid) d3 = -INFINITY;
     }
-    const float e0 = ex2_approx(d0), e1 = ex2_approx(d1), e2 = ex2_approx(d2), e3 = ex2_approx(d3);
+    float e0, e1, e2, e3;
+    if ((k / 4) % 4 < kExpFmaGroups) {   // compile-time per group: the loop is unrolled
+      ex2_fma2(d0, d1, e0, e1);
+      ex2_fma2(d2, d3, e2, e3);
+    } else {
+      e0 = ex2_approx(d0);
+      e1 = ex2_approx(d1);
+      e2 = ex2_approx(d2);
+      e3 = ex2_approx(d3);
+    }
     float l0, l1, l2, l3, h0, h1, h2, h3;
     fma2(l0, l1, e0, e1, kLo, kLo, kMag, kMag);
     fma2(l2, l3, e2, e3, kLo, kLo, kMag, kMag);
@@ -772,12 +830,13 @@ __global__ void __launch_bounds__(256) widen_kv_kernel(const __grid_constant__ I
 }
 
 // Exhaustive-check hook: the kernels' P-code function on an array.
+template <bool FMA>
 __global__ void pcode_kernel(const float* d, uint8_t* u, int64_t n, Int4Params p) {
   __shared__ float tau[16];
   if (threadIdx.x < 16) tau[threadIdx.x] = p.tau[threadIdx.x];
   __syncthreads();
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-    u[i] = static_cast<uint8_t>(pcode(d[i], tau));
+    u[i] = static_cast<uint8_t>(FMA ? pcode_fma(d[i], tau) : pcode(d[i], tau));
 }
 
 }  // namespace rota

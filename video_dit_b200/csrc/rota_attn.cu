@@ -831,15 +831,26 @@ rota_status rota_attn_get_error(void* stream) {
   return ROTA_OK;
 }
 
-rota_status rota_attn_debug_pcode(const float* dvals, uint8_t* u, int64_t n, void* stream) {
+static rota_status debug_pcode(bool fma, const float* dvals, uint8_t* u, int64_t n, void* stream) {
   if (n < 0 || (n > 0 && (!dvals || !u))) return ROTA_ERR_INVALID_ARG;
   if (n == 0) return ROTA_OK;
   rota::Int4Params p{};
   std::memcpy(p.tau, tau_table().tau, sizeof(p.tau));
   const int64_t blocks64 = (n + 255) / 256;
   const int blocks = static_cast<int>(blocks64 < 148 * 16 ? blocks64 : 148 * 16);
-  rota::pcode_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(dvals, u, n, p);
+  if (fma)
+    rota::pcode_kernel<true><<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(dvals, u, n, p);
+  else
+    rota::pcode_kernel<false><<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(dvals, u, n, p);
   return cuda_status(cudaGetLastError());
+}
+
+rota_status rota_attn_debug_pcode(const float* dvals, uint8_t* u, int64_t n, void* stream) {
+  return debug_pcode(false, dvals, u, n, stream);
+}
+
+rota_status rota_attn_debug_pcode_fma(const float* dvals, uint8_t* u, int64_t n, void* stream) {
+  return debug_pcode(true, dvals, u, n, stream);
 }
 
 rota_status rota_attn_debug_hadamard(int32_t n, int8_t* h) {

@@ -64,6 +64,7 @@ _SIGS = {
     "rota_attn_debug_dump_int4": ([_D, _BUF, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                    ctypes.c_int32, _P, _P, _P, _P], ctypes.c_int),
     "rota_attn_debug_pcode": ([_P, _P, ctypes.c_int64, _P], ctypes.c_int),
+    "rota_attn_debug_pcode_fma": ([_P, _P, ctypes.c_int64, _P], ctypes.c_int),
     "rota_attn_debug_inject_timeout": ([ctypes.c_int32, ctypes.c_uint64], ctypes.c_int),
     "rota_attn_debug_mma_cycles": ([ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P], ctypes.c_int),
     "rota_attn_fwd_int4_noalloc": ([_D, _P, _P, _P, _P, _P], ctypes.c_int),
@@ -225,6 +226,10 @@ def rota_attn_debug_dump_int4(desc, buffers, b, h, r0, nr, s_out, p_out, out, st
 
 def rota_attn_debug_pcode(d, u, stream=None) -> int:
     return _lib.rota_attn_debug_pcode(_ptr(d), _ptr(u), int(d.numel()), _stream(stream))
+
+
+def rota_attn_debug_pcode_fma(d, u, stream=None) -> int:
+    return _lib.rota_attn_debug_pcode_fma(_ptr(d), _ptr(u), int(d.numel()), _stream(stream))
 
 
 def rota_attn_debug_hadamard(n: int):
