@@ -42,6 +42,8 @@ CASES = {
                                        max_group=128),
     "row_sum_r1": synth.scaled(synth.WORKLOADS["wan480"], "r1", H=2, grid=(3, 10, 13), row_sum=1),
     "g128_r1_tiny": synth.scaled(synth.WORKLOADS["tiny"], "g128r1", max_group=128, row_sum=1),
+    # head_dim 64 with 8-channel blocks aligned to 16/24/24: the persistent prologue at d = 64
+    "tiny_had8": synth.scaled(synth.WORKLOADS["tiny"], "tiny_h8", had=(8, 8, 8)),
 }
 
 # Many key blocks per CTA (74), so every pipeline stage and barrier phase wraps many times.
@@ -201,15 +203,19 @@ def test_pcode_function_exhaustive_range(entry):
                                   want[bad[:5, 0]].cpu().numpy())
 
 
-def test_prologue_multi_unit_ranges_batch_and_flags():
-    """B = 2, H = 8, N = 1560 (25 blocks): 400 (batch, block, head) units, more
-    than the prologue's persistent CTAs, so CTAs take ranges of one or two
-    units that cross heads, blocks and the batch boundary; heads 3 and 6 are
+@pytest.mark.parametrize("base,B,H,grid", [("wan480", 2, 8, (4, 15, 26)), ("tiny", 2, 8, (3, 16, 14))])
+def test_prologue_multi_unit_ranges_batch_and_flags(base, B, H, grid):
+    """B = 2, H = 8, N = 1560 (25 blocks; d = 128) or N = 672 (11 blocks; d =
+    64): 400 / 176 (batch, block, head) units, so CTAs take ranges that cross
+    heads, blocks and the batch boundary (at d = 128 more units than the
+    persistent CTAs, so ranges of one or two units); heads 3 and 6 are
     flagged (their Q / K come out RoPE'd in fp16, their V job is skipped).
     Codes and scales of the INT4 heads and the RoPE'd rows of the flagged
     heads byte-exact against the oracle."""
     from gpu_util import desc_of, lib, to_dev
-    w = synth.scaled(synth.WORKLOADS["wan480"], "multi_unit", B=2, H=8, grid=(4, 15, 26))
+    had = (8, 8, 8) if base == "tiny" else None          # d = 64: blocks that fit a chunk
+    w = synth.scaled(synth.WORKLOADS[base], "multi_unit_" + base, B=B, H=H, grid=grid,
+                     **({"had": had} if had else {}))
     q, k, v = synth.make_inputs(w)
     flags = np.zeros(w.H, np.uint8)
     flags[[3, 6]] = 1

@@ -53,7 +53,8 @@ struct StreamSmem {
 struct ChunkRot {
   bool l1[4], l2[4], l3;
   float rn[4];
-  bool any2, any3;   // warp-uniform
+  bool any2, any3;   // warp-uniform: some lane has level 2 / 3
+  bool all1;         // warp-uniform: every lane has level 1 on all four pairs
 };
 
 __device__ __forceinline__ ChunkRot chunk_rot(const PrologueParams& p, int ch) {
@@ -74,6 +75,7 @@ __device__ __forceinline__ ChunkRot chunk_rot(const PrologueParams& p, int ch) {
   }
   c.any2 = __any_sync(0xffffffffu, any2);
   c.any3 = __any_sync(0xffffffffu, c.l3);
+  c.all1 = __all_sync(0xffffffffu, c.l1[0] && c.l1[1] && c.l1[2] && c.l1[3]);
   return c;
 }
 
@@ -86,8 +88,17 @@ __device__ __forceinline__ void rope_rotate8(float (&y)[8], float4 a0, float4 a1
   rope_pair(y[4], y[5], a1.x, a1.y);
   rope_pair(y[6], y[7], a1.z, a1.w);
   if (!rotate) return;
+  if (c.all1) {   // the level every lane takes on every pair: no selects
 #pragma unroll
-  for (int q = 0; q < 4; ++q) bfly(y[2 * q], y[2 * q + 1], c.l1[q]);
+    for (int q = 0; q < 4; ++q) {
+      const float u = y[2 * q], w = y[2 * q + 1];
+      y[2 * q] = __fadd_rn(u, w);
+      y[2 * q + 1] = __fsub_rn(u, w);
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) bfly(y[2 * q], y[2 * q + 1], c.l1[q]);
+  }
   if (c.any2) {
     bfly(y[0], y[2], c.l2[0]);
     bfly(y[1], y[3], c.l2[0]);
