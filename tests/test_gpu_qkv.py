@@ -25,6 +25,12 @@ CASES = {
     # HunyuanVideo 16/56/56 with 56-channel Hadamard blocks (the dense rotation pass), B = 2
     "hunyuan_h56": (synth.scaled(synth.WORKLOADS["hunyuan"], "qkv_hy", B=2, H=1, grid=(2, 5, 13),
                                  had=(16, 56, 56)), 192),
+    # H = 59, C = 1024: the heads' W rows (46 MB) exceed one raster group, so the
+    # kernel runs two groups, of 30 and 29 heads.  N = 26 (one ragged tile per
+    # head) keeps the oracle's projection short; outlier rows x4 keep the
+    # exact-grid sums below 2^24 units.
+    "wan_groups": (synth.scaled(synth.WORKLOADS["wan480"], "qkv_groups", H=59, grid=(1, 2, 13), qk_scale=4.0),
+                   1024),
 }
 
 
