@@ -18,6 +18,9 @@ TOL = 2e-3
 
 ONE = synth.Workload("one_token", B=1, H=2, d=64, rope_dim=(16, 24, 24), grid=(1, 1, 1))
 MAXH = synth.Workload("max_heads", B=1, H=256, d=64, rope_dim=(16, 24, 24), grid=(1, 2, 9))      # N=18
+# the same two shapes in the Wan layout (d = 128, Hadamard 4/2/2): the persistent prologue kernel
+ONE_WAN = synth.Workload("one_token_wan", B=1, H=2, d=128, rope_dim=(44, 42, 42), grid=(1, 1, 1))
+MAXH_WAN = synth.Workload("max_heads_wan", B=1, H=256, d=128, rope_dim=(44, 42, 42), grid=(1, 2, 9))
 SMALL = synth.scaled(synth.WORKLOADS["wan480"], "edge", H=2, grid=(2, 7, 11))                     # N=154
 
 
@@ -31,6 +34,10 @@ def _inputs(case):
         return ONE, synth.make_inputs(ONE, seed=7)
     if case == "max_heads":
         return MAXH, synth.make_inputs(MAXH, seed=8)
+    if case == "one_token_wan":
+        return ONE_WAN, synth.make_inputs(ONE_WAN, seed=7)
+    if case == "max_heads_wan":
+        return MAXH_WAN, synth.make_inputs(MAXH_WAN, seed=8)
     w = SMALL
     q, k, v = synth.make_inputs(w, seed=9)
     if case == "zeros":
@@ -50,7 +57,7 @@ def _inputs(case):
     raise KeyError(case)
 
 
-CASES = ["one_token", "max_heads", "zeros", "zero_k_block", "huge", "tiny_v"]
+CASES = ["one_token", "max_heads", "one_token_wan", "max_heads_wan", "zeros", "zero_k_block", "huge", "tiny_v"]
 
 
 @pytest.mark.parametrize("case", CASES)
@@ -78,7 +85,7 @@ def test_edge_case_parity(case):
         assert e <= TOL, (hh, e, rel, cos)
     if case == "zeros":
         assert not out.any()                       # every code 0: O = 0 exactly
-    if case == "one_token":
+    if case in ("one_token", "one_token_wan"):
         # one key: its P code is 15, so O = RN(RN(15 s v) / 15): two fp32
         # roundings away from the key's dequantised V row s v
         sv = ref["v_scale"][0, h, 0].astype(np.float64)
