@@ -32,10 +32,10 @@
 // One CTA = two 128-row query tiles of one head (256 rows), 512 threads:
 //   warp 0      TMA producer: the K and V^T images of each 64-key block
 //               -> a kOps-stage shared-memory ring;
-//   warp 1      issues S_t(j) = Q_t K_j^T for both tiles (128 x 64 each);
+//   warps 1, 3  issue S_t(j) = Q_t K_j^T (128 x 64), warp 1 for tile 0 and
+//               warp 3 (which also owns the TMEM allocation) for tile 1;
 //   warp 2      issues ACC^T = V_j^T P_t(j)^T for tile 0 then tile 1 into the
 //               one ACC^T buffer (128 channels x 128 queries);
-//   warp 3      owns the TMEM allocation;
 //   warps 4-7   softmax of tile 0, warps 8-11 of tile 1 (thread = query row
 //               = TMEM lane): running max, P codes into shared memory (the
 //               B operand of P V), the row sum of the codes, alpha;
@@ -111,8 +111,8 @@ struct Int4Smem {
   static constexpr int SPILL_BYTES = G == 128 ? 2 * kBM * kBN * 4 : 0;
   static constexpr int OFF_BAR = OFF_SPILL + SPILL_BYTES;
   // barriers: op_full[OPS] op_empty[OPS] q_full s_full[2] s_empty[2]
-  //           p_full[2][2] p_empty[2][2] acc_full acc_empty l_full mma_done[2]
-  static constexpr int NBAR = 2 * OPS + 1 + 2 + 2 + 4 + 4 + 1 + 1 + 1 + 2;
+  //           p_full[2][2] p_empty[2][2] acc_full acc_empty l_full mma_done[3]
+  static constexpr int NBAR = 2 * OPS + 1 + 2 + 2 + 4 + 4 + 1 + 1 + 1 + 3;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int BYTES = OFF_ABORT + 4;
@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* op_full = bars;
-  uint64_t* op_empty = bars + kOps;             // 2 arrivals: the S and the P V issuer's commits
+  uint64_t* op_empty = bars + kOps;             // 3 arrivals: the two S issuers' and the P V issuer's commits
   uint64_t* q_full = bars + 2 * kOps;           // 8 softmax warps staged their Q rows
   uint64_t* s_full = q_full + 1;                // [tile], commit
   uint64_t* s_empty = s_full + 2;               // [tile], 4 softmax warps hold S in registers
@@ -343,7 +343,7 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
   uint64_t* acc_full = p_empty + 4;             // commit of a P V
   uint64_t* acc_empty = acc_full + 1;           // 4 correction warps hold ACC in registers
   uint64_t* l_full = acc_empty + 1;             // 8 softmax warps wrote their rows' l
-  uint64_t* mma_done = l_full + 1;              // [2], one per issuing warp
+  uint64_t* mma_done = l_full + 1;              // [3], one per MMA-issuing warp (S tile 0, P V, S tile 1)
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + L::OFF_ABORT);
   float* sTau = reinterpret_cast<float*>(smem + L::OFF_TAU);
@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
   if (tid == 0) {
     for (int i = 0; i < kOps; ++i) {
       mbar_init(&op_full[i], 1);
-      mbar_init(&op_empty[i], 2);
+      mbar_init(&op_empty[i], 3);
     }
     mbar_init(q_full, 8);
     for (int t = 0; t < 2; ++t) {
@@ -377,8 +377,7 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 4);
     mbar_init(l_full, 8);
-    mbar_init(&mma_done[0], 1);
-    mbar_init(&mma_done[1], 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&mma_done[i], 1);
     *sAbort = 0;
     fence_mbar_init();
   }
@@ -418,9 +417,12 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       // drain: every issued copy has landed before the CTA may exit
       for (int j = (issued > kOps ? issued - kOps : 0); j < issued; ++j)
         warp_wait(&op_full[j % kOps], (j / kOps) & 1, lim);
-    } else if (warp == 1) {
-      // ---- S issuer: S_t(j) = Q_t K_j^T for t = 0, 1 (warp-uniform loop,
-      // one elected lane issues) ----
+    } else if (warp == 1 || warp == 3) {
+      // ---- S issuers: S_t(j) = Q_t K_j^T, warp 1 for tile 0 and warp 3 (after
+      // the TMEM allocation) for tile 1, so neither tile's next scores wait
+      // behind the other's (warp-uniform loop, one elected lane issues) ----
+      const int t = warp == 1 ? 0 : 1;
+      uint64_t* const done = &mma_done[t == 0 ? 0 : 2];
       constexpr uint32_t ID_S = idesc(1, 0, 0, kBM, kBN);   // e4m3 x e4m3 -> f32, 128 x 64
       const uint32_t hi_qk = sdesc_hi(L::SBO_QK, L::LAYOUT_QK);
       const uint32_t lo_q = sdesc_lo(smem_u32(smem + L::OFF_Q));
@@ -430,30 +432,28 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         const int op = j % kOps;
         if (!warp_wait(&op_full[op], (j / kOps) & 1, lim)) { ok = false; break; }
         const uint32_t lk = lo_op + op * (L::OP_BYTES >> 4);
-        for (int t = 0; t < 2; ++t) {
-          if (!warp_wait(&s_empty[t], (j & 1) ^ 1, lim)) { ok = false; break; }
-          tc_fence_after();
-          if (p.inject_skip && j == 0 && t == 0) continue;  // fault injection: never committed
-          const uint32_t lq = lo_q + t * (L::Q_BYTES >> 4);
-          const uint32_t d_s = tmem + L::T_S + t * kBN;
-          if (elect_one()) {
-            mma_f8f6f4_ss<0>(d_s, lq, hi_qk, lk, hi_qk, ID_S);
-#pragma unroll
-            for (int k = 1; k < D / 32; ++k) mma_f8f6f4_ss<1>(d_s, lq + 2 * k, hi_qk, lk + 2 * k, hi_qk, ID_S);
-            mma_commit(&s_full[t]);
-            // a commit tracks the MMAs of the thread that issues it: the
-            // stage's K tile is released by the lane that issued both tiles'
-            if (t == 1) mma_commit(&op_empty[op]);
-          }
+        if (!warp_wait(&s_empty[t], (j & 1) ^ 1, lim)) { ok = false; break; }
+        tc_fence_after();
+        if (p.inject_skip && j == 0 && t == 0) {   // fault injection: never committed
           __syncwarp();
+          continue;
         }
-        if (!ok) break;
+        const uint32_t lq = lo_q + t * (L::Q_BYTES >> 4);
+        const uint32_t d_s = tmem + L::T_S + t * kBN;
+        if (elect_one()) {
+          mma_f8f6f4_ss<0>(d_s, lq, hi_qk, lk, hi_qk, ID_S);
+#pragma unroll
+          for (int k = 1; k < D / 32; ++k) mma_f8f6f4_ss<1>(d_s, lq + 2 * k, hi_qk, lk + 2 * k, hi_qk, ID_S);
+          mma_commit(&s_full[t]);
+          mma_commit(&op_empty[op]);   // this tile's read of the stage's K tile
+        }
+        __syncwarp();
         if (warp_flag(sAbort)) { ok = false; break; }
       }
       if (!ok && lane == 0) *sAbort = 1;
-      if (elect_one()) mma_commit(&mma_done[0]);
+      if (elect_one()) mma_commit(done);
       __syncwarp();
-      warp_wait(&mma_done[0], 0, lim);
+      warp_wait(done, 0, lim);
     } else if (warp == 2) {
       // ---- P V issuer: ACC^T = V_j^T P_t(j)^T, tile 0 then tile 1, into
       // the one ACC^T buffer ----
