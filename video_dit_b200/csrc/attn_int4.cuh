@@ -35,10 +35,12 @@
 //   warps 1, 3  issue S_t(j) = Q_t K_j^T (128 x 64), warp 1 for tile 0 and
 //               warp 3 (which also owns the TMEM allocation) for tile 1;
 //   warp 2      issues ACC^T = V_j^T P_t(j)^T for tile 0 then tile 1 into the
-//               one ACC^T buffer (128 channels x 128 queries);
+//               one ACC^T buffer (128 channels x 128 queries); its commit
+//               also frees the P slot the MMA read;
 //   warps 4-7   softmax of tile 0, warps 8-11 of tile 1 (thread = query row
 //               = TMEM lane): running max, P codes into shared memory (the
-//               B operand of P V), the row sum of the codes, alpha;
+//               B operand of P V), the row sum of the codes, alpha (into a
+//               ring of its own, freed by the correction);
 //   warps 12-15 correction (thread = channel): O^T update per block, and the
 //               epilogue out = O / l.
 // TMEM (512 columns): S of tile t at 64 t, ACC^T at 128, O^T of tile t at
@@ -77,6 +79,14 @@ struct Int4Params {
 constexpr int kInt4Threads = 512;
 constexpr int kRowsPerCta = 2 * kBM;
 constexpr int kOps = 6;   // operand stages
+// The softmax may run kPSlots blocks ahead of the P V that reads its codes
+// and kAlphaRing blocks ahead of the correction that reads its alpha.  Both at
+// 2 measured fastest at 480p (alpha entries 1 / 2 / 3 / 4 / 8: 35.0 / 33.9 /
+// 34.9 / 34.6 / 34.4 ms; 3 P slots: +0.5 ms).  128-key groups emit block 2g + 1
+// before block 2g, so both need at least two entries.
+constexpr int kPSlots = 2;
+constexpr int kAlphaRing = 2;
+static_assert(kPSlots >= 2 && kAlphaRing >= 2, "a 128-key group emits its two blocks out of order");
 constexpr int kIssueRegs = 32;    // warps 0-3
 constexpr int kSoftmaxRegs = 128; // warps 4-11
 constexpr int kCorrRegs = 224;    // warps 12-15
@@ -102,17 +112,18 @@ struct Int4Smem {
   static constexpr int IMG_BYTES = OP_BYTES;      // one block in int4_work
   static constexpr int OFF_Q = 0;                                 // [tile]
   static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;               // [tile][slot]
-  static constexpr int OFF_OP = OFF_P + 4 * P_BYTES;              // [stage]
-  static constexpr int OFF_ALPHA = OFF_OP + OPS * OP_BYTES;       // float [tile][slot][128]
-  static constexpr int OFF_FLAG = OFF_ALPHA + 4 * kBM * 4;        // int [tile][slot][4 warps]
-  static constexpr int OFF_L = OFF_FLAG + 16 * 4;                 // float [tile][128]
+  static constexpr int OFF_OP = OFF_P + 2 * kPSlots * P_BYTES;    // [stage]
+  static constexpr int OFF_ALPHA = OFF_OP + OPS * OP_BYTES;       // float [tile][entry][128]
+  static constexpr int OFF_FLAG = OFF_ALPHA + 2 * kAlphaRing * kBM * 4;   // int [tile][entry][4 warps]
+  static constexpr int OFF_L = OFF_FLAG + 2 * kAlphaRing * 4 * 4;         // float [tile][128]
   static constexpr int OFF_TAU = OFF_L + 2 * kBM * 4;
   static constexpr int OFF_SPILL = OFF_TAU + 64;                  // float4 [tile][16][128] (G = 128)
   static constexpr int SPILL_BYTES = G == 128 ? 2 * kBM * kBN * 4 : 0;
   static constexpr int OFF_BAR = OFF_SPILL + SPILL_BYTES;
   // barriers: op_full[OPS] op_empty[OPS] q_full s_full[2] s_empty[2]
-  //           p_full[2][2] p_empty[2][2] acc_full acc_empty l_full mma_done[3]
-  static constexpr int NBAR = 2 * OPS + 1 + 2 + 2 + 4 + 4 + 1 + 1 + 1 + 3;
+  //           p_full[2][kPSlots] p_empty[2][kPSlots] acc_full acc_empty l_full
+  //           mma_done[3] a_full[2][kAlphaRing] a_empty[2][kAlphaRing]
+  static constexpr int NBAR = 2 * OPS + 1 + 2 + 2 + 4 * kPSlots + 1 + 1 + 1 + 3 + 4 * kAlphaRing;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int BYTES = OFF_ABORT + 4;
@@ -338,12 +349,14 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
   uint64_t* q_full = bars + 2 * kOps;           // 8 softmax warps staged their Q rows
   uint64_t* s_full = q_full + 1;                // [tile], commit
   uint64_t* s_empty = s_full + 2;               // [tile], 4 softmax warps hold S in registers
-  uint64_t* p_full = s_empty + 2;               // [tile][slot], 4 softmax warps wrote P, alpha
-  uint64_t* p_empty = p_full + 4;               // [tile][slot], 4 correction warps are done with them
-  uint64_t* acc_full = p_empty + 4;             // commit of a P V
+  uint64_t* p_full = s_empty + 2;               // [tile][slot], 4 softmax warps wrote the codes
+  uint64_t* p_empty = p_full + 2 * kPSlots;     // [tile][slot], commit of the P V that read them
+  uint64_t* acc_full = p_empty + 2 * kPSlots;   // commit of a P V
   uint64_t* acc_empty = acc_full + 1;           // 4 correction warps hold ACC in registers
   uint64_t* l_full = acc_empty + 1;             // 8 softmax warps wrote their rows' l
   uint64_t* mma_done = l_full + 1;              // [3], one per MMA-issuing warp (S tile 0, P V, S tile 1)
+  uint64_t* a_full = mma_done + 3;              // [tile][entry], 4 softmax warps wrote alpha and flags
+  uint64_t* a_empty = a_full + 2 * kAlphaRing;  // [tile][entry], 4 correction warps are done with them
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + L::OFF_ABORT);
   float* sTau = reinterpret_cast<float*>(smem + L::OFF_TAU);
@@ -370,14 +383,18 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       mbar_init(&s_full[t], 1);
       mbar_init(&s_empty[t], 4);
     }
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2 * kPSlots; ++i) {
       mbar_init(&p_full[i], 4);
-      mbar_init(&p_empty[i], 4);
+      mbar_init(&p_empty[i], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 4);
     mbar_init(l_full, 8);
     for (int i = 0; i < 3; ++i) mbar_init(&mma_done[i], 1);
+    for (int i = 0; i < 2 * kAlphaRing; ++i) {
+      mbar_init(&a_full[i], 4);
+      mbar_init(&a_empty[i], 4);
+    }
     *sAbort = 0;
     fence_mbar_init();
   }
@@ -464,19 +481,20 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       const uint32_t d_acc = tmem + L::T_ACC;
       bool ok = true;
       for (int j = 0; ok && j < nkb; ++j) {
-        const int op = j % kOps, sl = j & 1;
+        const int op = j % kOps, sl = j % kPSlots, pph = (j / kPSlots) & 1;
         if (!warp_wait(&op_full[op], (j / kOps) & 1, lim)) { ok = false; break; }
         const uint32_t lv = lo_v + op * (L::OP_BYTES >> 4);
         for (int t = 0; t < 2; ++t) {
           const int u = 2 * j + t;
-          if (!warp_wait(&p_full[2 * t + sl], (j >> 1) & 1, lim)) { ok = false; break; }
+          if (!warp_wait(&p_full[kPSlots * t + sl], pph, lim)) { ok = false; break; }
           if (!warp_wait(acc_empty, (u & 1) ^ 1, lim)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t lp = lo_p + (2 * t + sl) * (L::P_BYTES >> 4);
+          const uint32_t lp = lo_p + (kPSlots * t + sl) * (L::P_BYTES >> 4);
           if (elect_one()) {
             mma_f8f6f4_ss<0>(d_acc, lv, hi_64, lp, hi_64, ID_PV);
             mma_f8f6f4_ss<1>(d_acc, lv + 2, hi_64, lp + 2, hi_64, ID_PV);
             mma_commit(acc_full);
+            mma_commit(&p_empty[kPSlots * t + sl]);  // the tile's codes of block j are read
             if (t == 1) mma_commit(&op_empty[op]);   // the stage's V^T tile is read
           }
           __syncwarp();
@@ -550,17 +568,19 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     // the codes of block j -> its P slot (the B operand of P V), with alpha
     // (the factor on O before the block is added) and the warp's flag
     auto emit = [&](int j, const uint32_t (&pw)[kBN / 4], float alpha) -> bool {
-      const int sl = j & 1;
-      // the slot's previous codes (block j - 2) are consumed
-      if (j >= 2 && !warp_wait(&p_empty[2 * t + sl], ((j >> 1) & 1) ^ 1, lim)) return false;
-      uint8_t* sP = smem + L::OFF_P + (2 * t + sl) * L::P_BYTES;
+      const int ps = kPSlots * t + j % kPSlots, e = kAlphaRing * t + j % kAlphaRing;
+      // the slot's previous codes (block j - kPSlots) are read by their P V,
+      // and the entry's previous alpha (block j - kAlphaRing) by the correction
+      if (j >= kPSlots && !warp_wait(&p_empty[ps], ((j / kPSlots) & 1) ^ 1, lim)) return false;
+      if (j >= kAlphaRing && !warp_wait(&a_empty[e], ((j / kAlphaRing) & 1) ^ 1, lim)) return false;
+      uint8_t* sP = smem + L::OFF_P + ps * L::P_BYTES;
 #pragma unroll
       for (int i = 0; i < kBN / 16; ++i)
         *reinterpret_cast<uint4*>(sP + swz<64>(r, 16 * i)) =
             make_uint4(pw[4 * i], pw[4 * i + 1], pw[4 * i + 2], pw[4 * i + 3]);
-      sAlpha[(2 * t + sl) * kBM + r] = alpha;
+      sAlpha[e * kBM + r] = alpha;
       const bool moved = __any_sync(0xffffffffu, alpha != 1.f);
-      if (lane == 0) sFlag[(2 * t + sl) * 4 + (warp & 3)] = moved ? 1 : 0;
+      if (lane == 0) sFlag[e * 4 + (warp & 3)] = moved ? 1 : 0;
       if (dumping) {
         const int nvalid = min(kBN, p.N - j * kBN);
 #pragma unroll
@@ -571,7 +591,10 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[2 * t + sl]);
+      if (lane == 0) {
+        mbar_arrive(&p_full[ps]);
+        mbar_arrive(&a_full[e]);
+      }
       return true;
     };
     // alpha = 2^(m_old - m) for the rows whose max moved (exact 1 elsewhere; 0
@@ -677,9 +700,8 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     for (int j = 0; j < nkb && !aborted; ++j) {
       const float s18 = __fmul_rn(s_next, 262144.f);   // ACC = sum u v * 2^-18; exact scaling
       if (j + 1 < nkb && c < D) s_next = __ldg(vsc + (size_t)(j + 1) * D);
-      const int sl = j & 1;
       for (int t = 0; t < 2; ++t) {
-        const int u = 2 * j + t;
+        const int u = 2 * j + t, e = t * kAlphaRing + j % kAlphaRing;
         if (!warp_wait(acc_full, u & 1, lim)) { aborted = true; break; }
         tc_fence_after();
         const uint32_t tO = tmem + L::T_O + t * kBM + t_lane;
@@ -702,12 +724,12 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty);
-        // alpha and the flags of (tile t, block j): written before the codes
-        // the P V just used were released (already complete: no wait in effect)
-        if (!warp_wait(&p_full[2 * t + sl], (j >> 1) & 1, lim)) { aborted = true; break; }
-        const int* fl = sFlag + (2 * t + sl) * 4;
+        // alpha and the flags of (tile t, block j): written with the codes
+        // the P V just used (already complete: no wait in effect)
+        if (!warp_wait(&a_full[e], (j / kAlphaRing) & 1, lim)) { aborted = true; break; }
+        const int* fl = sFlag + e * 4;
         const bool moved = j > 0 && (fl[0] | fl[1] | fl[2] | fl[3]) != 0;
-        const float* al = sAlpha + (2 * t + sl) * kBM;
+        const float* al = sAlpha + e * kBM;
         // O in two 64-column halves (the first already loaded): FMAs, then two stores
         auto half = [&](int hb, uint32_t(&o)[64]) {
           if (j == 0) {
@@ -750,10 +772,10 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
           }
           half(1, o);
         }
-        // this tile's codes and alpha of block j are consumed (the O stores
+        // this tile's alpha and flags of block j are consumed (the O stores
         // may still be in flight: they are waited for before O is read again)
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_empty[2 * t + sl]);
+        if (lane == 0) mbar_arrive(&a_empty[e]);
       }
       if (warp_flag(sAbort)) aborted = true;
     }
