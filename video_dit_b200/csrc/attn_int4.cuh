@@ -270,7 +270,7 @@ __device__ __noinline__ uint32_t block_codes_exact(const uint32_t* sr, int nvali
 template <bool MASK, bool R1>
 __device__ __forceinline__ uint32_t block_codes(const uint32_t (&sr)[kBN], int nvalid, float c18, float m,
                                                 uint32_t (&pw)[kBN / 4], const float* tau, float& lsum) {
-  uint32_t sum_lo = 0, sum_hi = 0;
+  uint32_t usum = 0, sum_hi = 0;
   float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
   for (int k = 0; k < kBN; k += 4) {
@@ -298,23 +298,24 @@ __device__ __forceinline__ uint32_t block_codes(const uint32_t (&sr)[kBN], int n
     fma2(l2, l3, e2, e3, kLo, kLo, kMag, kMag);
     fma2(h0, h1, e0, e1, kHi, kHi, kMag, kMag);
     fma2(h2, h3, e2, e3, kHi, kHi, kMag, kMag);
-    sum_lo += __float_as_uint(l0) + __float_as_uint(l1) + __float_as_uint(l2) + __float_as_uint(l3);
     sum_hi += __float_as_uint(h0) + __float_as_uint(h1) + __float_as_uint(h2) + __float_as_uint(h3);
     pw[k / 4] = prmt(prmt(__float_as_uint(l0), __float_as_uint(l1), 0x0040u),
                      prmt(__float_as_uint(l2), __float_as_uint(l3), 0x0040u), 0x5410u);
+    usum = __dp4a(pw[k / 4], 0x01010101u, usum);   // the four codes' sum, from the packed word
     if (R1) {
       add2(ls0, ls1, ls0, ls1, e0, e1);
       add2(ls0, ls1, ls0, ls1, e2, e3);
     }
   }
   if (R1) lsum = __fmul_rn(15.f, __fadd_rn(ls0, ls1));
-  // 64 kMag bit patterns sum to 0xC0000000 (mod 2^32)
-  uint32_t usum = sum_lo - 0xC0000000u;
   // Exact decisions (rare): some key of the warp's rows lies in the band
   // where the two roundings differ, or a row's max is so large that its max
   // key could round past code 15.  Out of line, so that its registers do not
   // weigh on the main path.
-  const bool bad = (sum_lo != sum_hi) || !(fabsf(m) < kLogitBound);
+  // Each upper rounding is at least the lower one and 64 kMag bit patterns
+  // sum to 0xC0000000 (mod 2^32): the two agree on every key exactly when
+  // sum_hi - 0xC0000000 is the sum of the packed (lower) codes.
+  const bool bad = (sum_hi - 0xC0000000u != usum) || !(fabsf(m) < kLogitBound);
   if (__any_sync(0xffffffffu, bad)) {
     // copies made only here, so the scores stay in registers on the main path
     uint32_t s_copy[kBN], p_copy[kBN / 4];
