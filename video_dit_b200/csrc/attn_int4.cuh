@@ -543,15 +543,24 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     const bool dumping = p.s_dump != nullptr;   // kernel argument: uniform
     const bool dump_rows = dumping && row >= p.dbg_r0 && row < p.dbg_r0 + p.dbg_nr;
 
-    // S of block j -> registers; the buffer is released at once, so the MMA
-    // computes the tile's next scores while these are coded
-    auto load_s = [&](int j, uint32_t (&sr)[kBN]) -> bool {
+    // S of block j -> registers, in two parts: start_s waits for the scores
+    // and issues the TMEM loads, finish_s waits for the loads and releases the
+    // buffer at once, so the MMA computes the tile's next scores while these
+    // are coded.  With 64-key groups the next block's loads are started before
+    // this block's codes are emitted (sr is dead by then), so their latency
+    // overlaps the emit.
+    auto start_s = [&](int j, uint32_t (&sr)[kBN]) -> bool {
       if (!warp_wait(&s_full[t], j & 1, lim)) return false;
       tc_fence_after();
       uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
       uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
       tmem_ld32(tS, s0);
       tmem_ld32(tS + 32, s1);
+      return true;
+    };
+    auto finish_s = [&](int j, uint32_t (&sr)[kBN]) {
+      uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+      uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
       tmem_wait_dep2(s0, s1);
       tc_fence_before();
       __syncwarp();
@@ -564,6 +573,10 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
             p.s_dump[(size_t)(row - p.dbg_r0) * p.N + (size_t)j * kBN + k] =
                 static_cast<int32_t>(__uint_as_float(sr[k]) * 262144.f);
       }
+    };
+    auto load_s = [&](int j, uint32_t (&sr)[kBN]) -> bool {
+      if (!start_s(j, sr)) return false;
+      finish_s(j, sr);
       return true;
     };
     // the codes of block j -> its P slot (the B operand of P V), with alpha
@@ -617,11 +630,12 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
     float m = -INFINITY, l = 0.f;
     bool aborted = false;
     if constexpr (G == 64) {
-      for (int j = 0; j < nkb; ++j) {
+      uint32_t sr[kBN];
+      aborted = !start_s(0, sr);
+      for (int j = 0; j < nkb && !aborted; ++j) {
         const float c18 = c18_of(sk_next);
         if (j + 1 < nkb) sk_next = __ldg(ksc + j + 1);
-        uint32_t sr[kBN];
-        if (!load_s(j, sr)) { aborted = true; break; }
+        finish_s(j, sr);
         const int nvalid = min(kBN, p.N - j * kBN);
         const float smax = nvalid == kBN ? block_max<false>(sr, nvalid) : block_max<true>(sr, nvalid);
         const float m_old = m;
@@ -631,9 +645,11 @@ __global__ void __launch_bounds__(kInt4Threads, 1) attn_int4_kernel(const __grid
                                          : block_codes_l<true, R1>(sr, nvalid, c18, m, pw, sTau);
         const float alpha = alpha_of(j == 0, m_old, m);
         l = __fmaf_rn(l, alpha, lsum);
+        if (j + 1 < nkb && !start_s(j + 1, sr)) { aborted = true; break; }
         if (!emit(j, pw, alpha)) { aborted = true; break; }
         if (warp_flag(sAbort)) { aborted = true; break; }
       }
+      tmem_ld_wait();   // no TMEM load of this thread is left in flight
     } else {
       // 128-key groups: blocks j0 = 2g and j1 = 2g + 1 share the max over both,
       // so block j0's scores wait in shared memory while j1's come in; j1 is
