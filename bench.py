@@ -137,7 +137,7 @@ def workload_config(w, l2_note):
 # kernel on the F = 3 point (profiles/).  The traffic is the K/V images or
 # tiles and the output, linear in B * heads * N.  A kernel missing here has no
 # capture of its current version, and its traffic is reported as null.
-TRAFFIC_PER_HEAD_TOKEN = {"attn_int4_kernel": 771.8, "attn_fp16_kernel": 1076.75}
+TRAFFIC_PER_HEAD_TOKEN = {"attn_int4_kernel": 772.2, "attn_fp16_kernel": 1076.75}
 
 
 def traffic_per_launch(kernel, w, heads):

@@ -80,12 +80,12 @@ constexpr int kInt4Threads = 512;
 constexpr int kRowsPerCta = 2 * kBM;
 constexpr int kOps = 6;   // operand stages
 // The softmax may run kPSlots blocks ahead of the P V that reads its codes
-// and kAlphaRing blocks ahead of the correction that reads its alpha.  Both at
-// 2 measured fastest at 480p (alpha entries 1 / 2 / 3 / 4 / 8: 35.0 / 33.9 /
-// 34.9 / 34.6 / 34.4 ms; 3 P slots: +0.5 ms).  128-key groups emit block 2g + 1
-// before block 2g, so both need at least two entries.
+// and kAlphaRing blocks ahead of the correction that reads its alpha.
+// Measured at 480p: alpha entries 2 / 3 / 4 / 5 / 6 take 32.6 / 32.0 / 32.7 /
+// 32.0 / 31.9 ms, and a third P slot adds 0.7 ms.  128-key groups emit block
+// 2g + 1 before block 2g, so both need at least two entries.
 constexpr int kPSlots = 2;
-constexpr int kAlphaRing = 2;
+constexpr int kAlphaRing = 3;
 static_assert(kPSlots >= 2 && kAlphaRing >= 2, "a 128-key group emits its two blocks out of order");
 constexpr int kIssueRegs = 32;    // warps 0-3
 constexpr int kSoftmaxRegs = 128; // warps 4-11
