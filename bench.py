@@ -136,12 +136,16 @@ def workload_config(w, l2_note):
 # (B=1, H=40, N=17160, whose output and operand images exceed L2), the FP16
 # kernel on the F = 3 point (profiles/).  The traffic is the K/V images or
 # tiles and the output, linear in B * heads * N.  A kernel missing here has no
-# capture of its current version, and its traffic is reported as null.
+# capture of its current version, and its traffic is reported as null; so is
+# the INT4 kernel's for the P-code variants (max group 128, R1 row sum), whose
+# instantiations were not captured.
 TRAFFIC_PER_HEAD_TOKEN = {"attn_int4_kernel": 772.2, "attn_fp16_kernel": 1076.75}
 
 
 def traffic_per_launch(kernel, w, heads):
     per = TRAFFIC_PER_HEAD_TOKEN.get(kernel)
+    if kernel == "attn_int4_kernel" and (w.max_group not in (0, 64) or w.row_sum):
+        per = None
     return None if per is None or heads == 0 else per * w.B * heads * w.N
 
 

@@ -101,6 +101,9 @@ WORKLOADS = {
 # as one Hadamard block (Paley I, q = 43) and the 56-channel ones (Paley II, q = 13, doubled)
 WORKLOADS["wan480_h44"] = dataclasses.replace(WORKLOADS["wan480"], name="wan480_h44", had=(44, 2, 2))
 WORKLOADS["hunyuan_h56"] = dataclasses.replace(WORKLOADS["hunyuan"], name="hunyuan_h56", had=(16, 56, 56))
+# the P-code numerics variants on the 480p recipe: one max per 128 keys, and the R1 row sum
+WORKLOADS["wan480_g128"] = dataclasses.replace(WORKLOADS["wan480"], name="wan480_g128", max_group=128)
+WORKLOADS["wan480_r1"] = dataclasses.replace(WORKLOADS["wan480"], name="wan480_r1", row_sum=1)
 for _F in (3, 6, 11, 21, 31):
     WORKLOADS[f"sweep{_F}"] = Workload(f"sweep{_F}", B=1, H=40, grid=(_F, 30, 52), **_WAN)
     WORKLOADS[f"sweep{_F}_fp16"] = Workload(f"sweep{_F}_fp16", B=1, H=40, grid=(_F, 30, 52),
